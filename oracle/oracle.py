@@ -54,6 +54,8 @@ def lib():
         L.pwo_attn_grouped.argtypes = [p, p, p, p, C.c_int, p, C.c_int, C.c_int, C.c_int, C.c_int,
                                        p, f64, f64, f64, p, p, p, p, p, i64, C.c_int, C.c_int, p]
         L.pwo_attn_grouped.restype = C.c_int
+        L.pwo_double_to_bf16_n.argtypes = [p, p, i64]
+        L.pwo_double_to_bf16_n.restype = None
         _lib = L
     return _lib
 
@@ -85,10 +87,21 @@ def bf16_to_f64(bits) -> np.ndarray:
 def f64_to_bf16(x) -> np.ndarray:
     """binary64 -> bf16 bits, round to nearest even (elementwise through the C routine)."""
     L = lib()
-    x = np.asarray(x, dtype=np.float64)
-    flat = np.fromiter((L.pwo_double_to_bf16(float(v)) for v in x.ravel()), dtype=np.uint16,
-                       count=x.size)
-    return flat.reshape(x.shape)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, np.uint16)
+    L.pwo_double_to_bf16_n(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """bf16 bits -> binary64 values (exact), vectorised through a 65536-entry table."""
+    global _BF16_TABLE
+    if _BF16_TABLE is None:
+        _BF16_TABLE = bf16_to_f64(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    return _BF16_TABLE[np.asarray(bits, dtype=np.uint16)]
+
+
+_BF16_TABLE = None
 
 
 # ---- grouping ------------------------------------------------------------------------------

@@ -447,3 +447,10 @@ int pwo_attn_grouped(const uint16_t *Q, const uint8_t *K, const uint8_t *V,
     }
     return PWO_OK;
 }
+
+/* Elementwise pwo_double_to_bf16 over an array (same rounding, one call). */
+void pwo_double_to_bf16_n(const double *x, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = pwo_double_to_bf16(x[i]);
+}

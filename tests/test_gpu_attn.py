@@ -1,0 +1,120 @@
+"""pw_attn on the GPU against the oracle, element by element.
+
+Small cases compare every output row; the benchmark workloads at full size compare every row
+(workloads 1-2) or a sample of rows the oracle computes one by one (workloads 3-5), always in
+the same launch configuration the benchmark times (pw_group then pw_attn on one stream).
+"""
+import numpy as np
+import pytest
+import torch
+
+from dynamic_sparse_attention_pw_b200 import api, synth
+from oracle import oracle
+
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, W, g):
+    d = api.device_inputs(inp)
+    status = api.new_status()
+    O, gr = api.prefill(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["sel_pages"],
+                        d["cu_seqlens"], d["cu_seqlens_host"], W, g, k_scale=d["k_scale"],
+                        v_scale=d["v_scale"], sm_scale=d["sm_scale"], status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return O.view(torch.int16).cpu().numpy().view(np.uint16), gr
+
+
+def _small(seed, seqlens, Hq, Hkv, kmax, selection="uniform", **kw):
+    return synth.Workload(f"gpu-attn{seed}", 400 + seed, tuple(seqlens), Hq=Hq, Hkv=Hkv,
+                          kmax=kmax, selection=selection, **kw)
+
+
+SMALL = [
+    # (workload, W, g): ragged batch, GQA 3, tile of 24 rows
+    (_small(1, [200, 64, 1, 130], 6, 2, 5, shuffled_pages=True), 16, 8),
+    # 64-row tiles, several union pages
+    (_small(2, [1024], 8, 1, 6, "fixed2"), 32, 8),
+    # full 128-row tile (g=16, G=8)
+    (_small(3, [512], 16, 2, 6, "community", communities=3), 32, 16),
+    # one query per group, contiguous groups
+    (_small(4, [300, 77], 4, 1, 8), 1, 1),
+    (_small(5, [300, 77], 4, 2, 8, shuffled_pages=True), 8, 8),
+    # ragged tails and long unions (every earlier page selected)
+    (_small(6, [70, 129, 300], 4, 1, 8), 24, 8),
+    (_small(7, [2048], 8, 1, 32, "uniform"), 64, 8),
+    # tile rows not a multiple of 32 and g not a power of two
+    (_small(8, [450], 10, 2, 7, "community", communities=2), 30, 6),
+]
+
+
+@pytest.mark.parametrize("wl,W,g", SMALL)
+def test_attn_matches_oracle_small(wl, W, g):
+    inp = parity.inputs(wl)
+    got, _ = _run(inp, W, g)
+    ref = oracle.attn_all(inp)
+    parity.compare_rows(got.reshape(-1, 128), ref.reshape(-1, 128), wl.name)
+
+
+def test_dense_causal_selection_long_unions():
+    # Every token selects all of its causal pages: unions of up to 32 pages, the running max
+    # moves often, so the lazy rescale of O is exercised.
+    T, Hkv = 2048, 1
+    wl = _small(9, [T], 8, Hkv, 32)
+    inp = dict(parity.inputs(wl))
+    sel = np.full((T, Hkv, 32), -1, np.int32)
+    for t in range(T):
+        o = t // 64
+        sel[t, 0, : o + 1] = np.arange(o + 1)
+    inp["sel_pages"] = sel
+    got, _ = _run(inp, 64, 8)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128), "dense")
+
+
+@pytest.mark.parametrize("qscale", [1e-6, 1.0, 3000.0])
+def test_query_magnitudes_and_scales(qscale):
+    wl = _small(10, [640, 200], 8, 2, 6, shuffled_pages=True)
+    inp = dict(parity.inputs(wl))
+    q = torch.from_numpy(inp["Q"].view(np.int16)).view(torch.bfloat16).float() * qscale
+    inp["Q"] = q.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    inp["k_scale"], inp["v_scale"] = 0.75, 1.5
+    inp["sm_scale"] = inp["sm_scale"] / max(qscale, 1.0) ** 0.5
+    got, _ = _run(inp, 32, 8)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128),
+                        f"qscale {qscale}")
+
+
+def test_empty_selections_give_zero_rows():
+    wl = _small(11, [300], 4, 1, 6)
+    inp = dict(parity.inputs(wl))
+    sel = inp["sel_pages"].copy()
+    sel[100:140] = -1          # 40 tokens select nothing
+    inp["sel_pages"] = sel
+    got, _ = _run(inp, 32, 8)
+    assert np.all(got.reshape(wl.T, wl.Hq, 128)[100:140] == 0)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128), "empty")
+
+
+@pytest.mark.parametrize("cfg,W", [(1, 32), (2, 64)])
+def test_attn_full_workload_every_row(cfg, W):
+    wl = synth.WORKLOADS[cfg]
+    inp = parity.inputs(wl)
+    got, _ = _run(inp, W, wl.g)
+    ref = oracle.attn_all(inp)
+    parity.compare_rows(got.reshape(-1, 128), ref.reshape(-1, 128), wl.name)
+
+
+@pytest.mark.parametrize("cfg,W,g", [(3, 128, 8), (3, 8, 8), (3, 128, 1), (4, 128, 8),
+                                     (4, 256, 8), (5, 128, 8)])
+def test_attn_full_workload_sampled_rows(cfg, W, g):
+    wl = synth.WORKLOADS[cfg]
+    inp = parity.inputs(wl)
+    got, gr = _run(inp, W, g)
+    gh = gr.to_host()
+    parity.assert_groups_equal(gh, parity.oracle_groups(wl, W, g))
+    rt, rh = parity.sample_rows(wl, gh, n_random=3000, seed=cfg)
+    ref = oracle.attn_rows(inp, rt, rh)
+    got = got.reshape(wl.T, wl.Hq, 128)[rt, rh]
+    parity.compare_rows(got, ref, f"{wl.name} W={W} g={g}")
