@@ -141,6 +141,30 @@ pw_status pw_attn(const void *Q, const void *K_pages, const void *V_pages,
                   float k_scale, float v_scale, float sm_scale,
                   const pw_groups *groups, void *O, int32_t *dev_status, void *stream);
 
+/* pw_group without a caller-supplied workspace.  The paper has no counterpart: this is a
+ * convenience of this library for callers that cannot allocate device memory, e.g. code running
+ * where cudaMalloc is not allowed (it can synchronise the device) or a plug-in whose host
+ * application owns the whole memory budget and hands it only input and output buffers.
+ *
+ * Same arguments, outputs and errors as pw_group, minus workspace / workspace_bytes.  The
+ * scratch is a fixed device array of PW_NOALLOC_SCRATCH_BYTES inside the library; every GPU that
+ * loads the library holds it until the process exits.  The call itself allocates nothing (no
+ * cudaMalloc, no cudaFree, no allocating library routine).
+ *   - Shapes whose workspace (pw_groups_size) exceeds PW_NOALLOC_SCRATCH_BYTES are rejected
+ *     with PW_ERR_CAPACITY before any device work; use pw_group with your own workspace then.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream capture.
+ *     The stream must belong to the current device.
+ *   - All calls on a device share the one array, which keeps the last call's contents.  Nothing
+ *     in it needs clearing between calls, but calls that overlap on the GPU (different streams,
+ *     no ordering between them) race on it and must not be issued.
+ */
+#define PW_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+pw_status pw_group_noalloc(const int32_t *sel_pages, const int32_t *cu_seqlens,
+                           const int32_t *cu_seqlens_host, int B, int Hkv, int kmax, int W, int g,
+                           const pw_groups *groups, int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
