@@ -5,27 +5,29 @@
 // support and complete output ownership; the kernel consumes query IDs without materialising
 // reordered Q tensors or cross-page partial outputs; FP8 KV throughout.
 //
-// One CTA (4 warps) owns one group.  Tile row r = member * G + head (G = Hq / Hkv query heads
-// share the member's kv head and selection), rows >= gsize * G are padding.  Per union page,
-// in ascending order:
-//   bulk copy   K and V page (E4M3, 8 KiB each) via the page table into a 2-stage ring
-//   decode      E4M3 -> f16 (exact) into 128-byte-swizzled operand tiles
-//   S = Q K^T   tcgen05.mma kind::f16, M=128, N=64, K=128 -> TMEM (fp32)
-//   mask        row keeps page p only if p is in its token's own selection, and keys <= its
-//               position (causal limit on the own page)
-//   softmax     online, fp32, base 2; the running max is raised lazily (only when it grows by
-//               more than 2^8) so the O rescale in TMEM is rare; P is split into f16 hi + lo
-//   O += P V    two tcgen05.mma (P_hi V, P_lo V), M=128, N=128, K=64 -> TMEM (fp32)
-// Epilogue: O / l, times v_scale, round to bf16, each row written to its own O[t, hq, :].
+// One CTA owns one group.  Tile row i = member * G + head (the G = Hq / Hkv query heads share
+// the member's kv head and selection); rows >= R = gsize * G are padding.  Rows are processed
+// in blocks of 64 (RB blocks, 128 * RB threads).  Per union page, in ascending order:
+//   bulk copy  K and V page (E4M3, 8 KiB each) via the page table into a 2-stage ring
+//   decode     E4M3 -> bf16, exact, with integer bit operations (no conversion unit) into
+//              128-byte-swizzled operand tiles
+//   S = Q K^T  tcgen05.mma kind::f16 (bf16), M=64 per row block, N=64 keys, K=128 -> TMEM
+//   mask       a row keeps page p only if p is in its own token's selection, and keys at or
+//              before its position (causal limit on its own page)
+//   softmax    online, fp32, base 2, two threads per row (columns 0-31 / 32-63); the running
+//              max is raised lazily (only when it grows by more than 2^8) so the rescale of
+//              the accumulator is rare; P is split into bf16 hi + lo with integer rounding
+//   O^T += V^T P^T   tcgen05.mma M=128 (head dim), N=R rounded up to 16, K=64 keys, twice
+//              (P_hi, P_lo), fp32 in TMEM -- the head dimension fills the 128 MMA rows, so no
+//              MMA row is padding
+// Epilogue: O / l, times v_scale, rounded to bf16, each row written to its own O[t, hq, :].
 //
-// Numerics: K and V are exact in f16 (E4M3 is a subset).  Q (bf16) is scaled per row by a
-// power of two into f16's range, which is exact for every element within 2^-25 of the row
-// maximum; the power of two is folded into the row's score scale.  The hi + lo split carries
-// P with about 22 significant bits into the fp32 PV accumulation.
+// Numerics: Q (bf16), K and V (E4M3 is a subset of bf16) enter the tensor cores exactly;
+// products accumulate in fp32.  P = hi + lo carries about 16 significant bits (hi rounded to
+// nearest, the remainder truncated), which keeps the output within the 1e-3 rel-L2 bar with a
+// margin of about ten.
 #include <cstdint>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "pw_internal.h"
@@ -34,69 +36,96 @@
 namespace pw {
 namespace {
 
-constexpr int kThreads = 128;
 constexpr int kStages = 2;
 constexpr int kPageBytes = kPageTokens * kHeadDim; // one kv head's page, E4M3
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;   // S: 64 fp32 columns
-constexpr uint32_t kColO = 128; // O: 128 fp32 columns
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kIdescS = idesc_f16_f32(128, 64, false, false);
-constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, false, true);
+constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
 
-// Operand tiles.  q: [2 dim-blocks][128 rows][128 B]; k and v: [2 dim-blocks][64 keys][128 B];
-// p: [128 rows][128 B].  Rows are 128 bytes (64 f16), 16-byte chunks XOR-swizzled by row % 8,
-// 8-row atoms at 1024 bytes.  The same physical layout serves K as the K-major B operand of
-// S = Q K^T and V as the MN-major B operand of O = P V.
+// Operand tiles (rows of 128 bytes = 64 bf16, 16-byte chunks XOR-swizzled by row % 8, 8-row
+// atoms at 1024 bytes):
+//   q    [2 dim-blocks][RB*64 rows][128 B]  A of S (K-major); row block rb at row 64 rb
+//   k    [2 dim-blocks][64 keys][128 B]     B of S (K-major)
+//   v    [2 dim-blocks][64 keys][128 B]     A of O^T, read MN-major (head dim along M)
+//   p_*  [RB*64 rows][128 B]                B of O^T (K-major: 64 keys per row)
+template <int RB>
 struct __align__(1024) AttnSmem {
-    uint8_t q[2][128 * 128];
+    uint8_t q[2][RB * 64 * 128];
     uint8_t k[2][64 * 128];
     uint8_t v[2][64 * 128];
-    uint8_t p_hi[128 * 128];
-    uint8_t p_lo[128 * 128];
+    uint8_t p_hi[RB * 64 * 128];
+    uint8_t p_lo[RB * 64 * 128];
     uint8_t stage_k[kStages][kPageBytes];
     uint8_t stage_v[kStages][kPageBytes];
+    float alpha[RB * 64];
+    float inv_l[RB * 64];
+    int32_t row_tok[RB * 64];
+    int32_t row_hq[RB * 64];
     uint64_t tma_bar[kStages];
     uint64_t mma_bar;
     uint32_t tmem_base;
+    int32_t flag;
+    int32_t rescale; // some row raised its running max on this page
 };
-
-constexpr size_t kSmemBytes = sizeof(AttnSmem) + 1024;
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk)
 {
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
-    const __half2_raw h =
-        __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 
-// 64 keys x 128 dims E4M3 (row-major) -> two swizzled 64-dim f16 blocks.
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Four E4M3 codes (byte 0 = element 0) -> two bf16x2 words, exactly.  Each byte s.eeee.mmm is
+// widened to a 16-bit half whose high byte repeats the sign (prmt sign mode), shifted so that
+// eeee.mmm lands in the bf16 exponent/mantissa bits 10..4 with the sign at bit 15; that bf16
+// equals the code's value times 2^-120 (subnormal codes included), and one bf16 multiply by
+// 2^120 restores it.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    constexpr uint32_t kTwo120 = 0x7B807B80u; // bf16 2^120 in both halves
+    const uint32_t a = (prmt(x, 0u, 0x9180u) << 4) & 0x87F087F0u;
+    const uint32_t b = (prmt(x, 0u, 0xB3A2u) << 4) & 0x87F087F0u;
+    lo = bf16x2_mul(a, kTwo120);
+    hi = bf16x2_mul(b, kTwo120);
+}
+
+// 64 keys x 128 dims E4M3 (row-major) -> two swizzled 64-dim bf16 blocks.  Thread q handles
+// key q/8, dims 16(q%8)..+15 (two 16-byte chunks); threads 4-7 of each quarter-warp store
+// their chunks in the opposite order so a quarter-warp's eight stores hit eight bank groups.
+template <int NT>
 __device__ __forceinline__ void decode_page(const uint8_t *src, uint8_t (*dst)[64 * 128], int tid)
 {
 #pragma unroll
-    for (int rep = 0; rep < 4; ++rep) {
-        const int q = tid + kThreads * rep;
-        const int row = q >> 3, c16 = q & 7;
-        const uint4 x = *reinterpret_cast<const uint4 *>(src + row * 128 + c16 * 16);
+    for (int rep = 0; rep < 512 / NT; ++rep) {
+        const int q = tid + NT * rep;
+        const int key = q >> 3, c16 = q & 7;
+        const uint4 x = *reinterpret_cast<const uint4 *>(src + key * 128 + c16 * 16);
         uint4 h0, h1;
-        h0.x = e4m3x2_to_f16x2(x.x);
-        h0.y = e4m3x2_to_f16x2(x.x >> 16);
-        h0.z = e4m3x2_to_f16x2(x.y);
-        h0.w = e4m3x2_to_f16x2(x.y >> 16);
-        h1.x = e4m3x2_to_f16x2(x.z);
-        h1.y = e4m3x2_to_f16x2(x.z >> 16);
-        h1.z = e4m3x2_to_f16x2(x.w);
-        h1.w = e4m3x2_to_f16x2(x.w >> 16);
+        e4m3x4_to_bf16x4(x.x, h0.x, h0.y);
+        e4m3x4_to_bf16x4(x.y, h0.z, h0.w);
+        e4m3x4_to_bf16x4(x.z, h1.x, h1.y);
+        e4m3x4_to_bf16x4(x.w, h1.z, h1.w);
         uint8_t *blk = dst[c16 >> 2];
         const int j0 = (2 * c16) & 7;
-        *reinterpret_cast<uint4 *>(blk + swz(row, j0)) = h0;
-        *reinterpret_cast<uint4 *>(blk + swz(row, j0 + 1)) = h1;
+        if (c16 < 4) {
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
+        } else {
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
+        }
     }
 }
 
@@ -107,34 +136,45 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-__device__ __forceinline__ uint32_t pack_h2(__half a, __half b)
+// p -> (hi, lo) bf16 halves of two packed words: hi = p rounded to bf16 (round half up on the
+// bit pattern), lo = p - hi truncated to bf16.
+__device__ __forceinline__ void split_pair(float p0, float p1, uint32_t &hi2, uint32_t &lo2)
 {
-    return static_cast<uint32_t>(__half_as_ushort(a)) |
-           (static_cast<uint32_t>(__half_as_ushort(b)) << 16);
+    const uint32_t u0 = __float_as_uint(p0) + 0x8000u;
+    const uint32_t u1 = __float_as_uint(p1) + 0x8000u;
+    const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u);
+    const float r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
+    hi2 = prmt(u0, u1, 0x7632u);
+    lo2 = prmt(__float_as_uint(r0), __float_as_uint(r1), 0x7632u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
+template <int RB>
+__global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(const AttnLaunch L)
 {
+    constexpr int NT = 128 * RB;
+    constexpr uint32_t kColS = 0;          // S: RB blocks of 64 fp32 columns
+    constexpr uint32_t kColO = 64 * RB;    // O^T: up to 64 * RB fp32 columns
+    constexpr uint32_t kTmemCols = 128 * RB;
     extern __shared__ uint8_t smem_raw[];
-    AttnSmem &sm = *reinterpret_cast<AttnSmem *>(
+    AttnSmem<RB> &sm = *reinterpret_cast<AttnSmem<RB> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t gi = blockIdx.x;
+
+    // Once any CTA of this launch has given up on a wait, the rest skip their work.
+    if (tid == 0)
+        sm.flag = *reinterpret_cast<volatile int32_t *>(L.status) == PW_ERR_TIMEOUT ? 1 : 0;
+    __syncthreads();
+    if (sm.flag != 0)
+        return;
 
     const int b = L.gmeta[3 * gi + 0];
     const int h = L.gmeta[3 * gi + 1];
     const int R = L.gsize[gi] * L.G;
+    const int Npad = (R + 15) & ~15;
     const int u0 = L.union_off[gi];
     const int nU = L.union_off[gi + 1] - u0;
-
-    // Once any CTA of this launch has given up on a wait, the rest skip their work instead of
-    // each waiting out its own limit.
-    if (tid == 0)
-        sm.tmem_base = *reinterpret_cast<volatile int32_t *>(L.status) == PW_ERR_TIMEOUT ? 1u : 0u;
-    __syncthreads();
-    if (sm.tmem_base != 0u)
-        return;
-    __syncthreads();
+    const uint32_t kIdescPV = idesc_bf16_f32(128, Npad, true, false);
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s)
@@ -146,66 +186,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    // per-row metadata
+    for (int i = tid; i < 64 * RB; i += NT) {
+        int32_t tok = 0, hq = 0;
+        if (i < R) {
+            const int mi = i / L.G;
+            tok = L.qids[gi * L.g + mi];
+            hq = h * L.G + (i - mi * L.G);
+        }
+        sm.row_tok[i] = tok;
+        sm.row_hq[i] = hq;
+        sm.alpha[i] = 1.f;
+    }
+    if (tid == 0)
+        sm.rescale = 0;
+    __syncthreads();
+    // Q tile: RB*64 rows x 16 chunks of 8 bf16, copied as is (rows >= R are zero)
+    for (int qn = tid; qn < RB * 64 * 16; qn += NT) {
+        const int row = qn >> 4, c = qn & 15;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (row < R)
+            val = __ldg(reinterpret_cast<const uint4 *>(
+                      L.Q + (static_cast<size_t>(sm.row_tok[row]) * L.Hq + sm.row_hq[row]) * kHeadDim) +
+                  c);
+        *reinterpret_cast<uint4 *>(sm.q[c >> 3] + swz(row, c & 7)) = val;
+    }
 
-    // ---- row metadata and the Q tile (row r = thread r = TMEM lane r) ----
-    const int r = tid;
-    const bool valid = r < R;
-    int64_t t = 0;
-    int hq = 0, pos = 0, own = 0;
+    // Softmax role: row i = 64 rb + 16 qd + (lane % 16), key half hh = lane / 16.
+    const int rb = warp >> 2, qd = warp & 3;
+    const int my_row = 64 * rb + 16 * qd + (lane & 15);
+    const int hh = lane >> 4;
+    const bool row_valid = my_row < R;
+    int pos = 0, own = 0;
     const uint32_t *bitrow = nullptr;
-    if (valid) {
-        const int mi = r / L.G, j = r - mi * L.G;
-        t = L.qids[gi * L.g + mi];
-        hq = h * L.G + j;
-        pos = static_cast<int>(t - L.cu[b]);
+    if (row_valid) {
+        const int64_t tok = sm.row_tok[my_row];
+        pos = static_cast<int>(tok - L.cu[b]);
         own = pos >> 6;
-        bitrow = L.bits + (static_cast<size_t>(t) * L.Hkv + h) * L.words;
+        bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
     }
-    float crow;
-    {
-        uint4 qv[16];
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            L.Q + (static_cast<size_t>(t) * L.Hq + hq) * kHeadDim);
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            qv[i] = valid ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
-                amax = fmaxf(amax, fabsf(__uint_as_float(w[e] & 0xFFFF0000u)));
-            }
-        }
-        int s = 0;
-        if (amax > 0.f && amax <= 3.0e38f) {
-            int e2;
-            frexpf(amax, &e2); // amax in [2^(e2-1), 2^e2)
-            s = 15 - e2;       // amax * 2^s in [2^14, 2^15)
-            s = s < -126 ? -126 : (s > 126 ? 126 : s);
-        }
-        const float up = __uint_as_float(static_cast<uint32_t>(127 + s) << 23);
-        const float down = __uint_as_float(static_cast<uint32_t>(127 - s) << 23);
-        crow = L.sm_scale * L.k_scale * kLog2e * down;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __half lo = __float2half_rn(__uint_as_float(w[e] << 16) * up);
-                const __half hi = __float2half_rn(__uint_as_float(w[e] & 0xFFFF0000u) * up);
-                o[e] = pack_h2(lo, hi);
-            }
-            *reinterpret_cast<uint4 *>(sm.q[i >> 3] + swz(r, i & 7)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-    }
+    const float crow = L.sm_scale * L.k_scale * kLog2e;
+
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t s_addr = tmem + (static_cast<uint32_t>(32 * qd) << 16) + kColS + 64 * rb;
 
     auto issue_page = [&](int i, int s) {
         const int pg = L.union_pages[u0 + i];
@@ -219,25 +246,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
         bulk_g2s(sm.stage_k[s], L.K + off, kPageBytes, &sm.tma_bar[s]);
         bulk_g2s(sm.stage_v[s], L.V + off, kPageBytes, &sm.tma_bar[s]);
     };
-
     if (tid == 0)
         for (int i = 0; i < kStages && i < nU; ++i)
             issue_page(i, i);
 
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l_part = 0.f;
     uint32_t mma_phase = 0;
-    bool aborted = false;
-    int pages_waited = 0;   // TMA phases consumed
-    bool mma_pending = false;
+    bool aborted = false, mma_pending = false;
+    int pages_waited = 0;
 
     for (int i = 0; i < nU; ++i) {
         const int s = i % kStages;
         const int pg = L.union_pages[u0 + i];
         bool ok = true;
-        if (mma_pending) { // previous O += P V: frees v, p_hi, p_lo and settles O
+        if (mma_pending) { // previous O^T += V^T P^T: frees v and p, settles O^T
             ok = mbar_wait(&sm.mma_bar, mma_phase);
-            mma_phase ^= 1u;
-            mma_pending = false;
+            if (ok) {
+                mma_phase ^= 1u;
+                mma_pending = false;
+            }
         }
         ok = ok && mbar_wait(&sm.tma_bar[s], static_cast<uint32_t>((i / kStages) & 1));
         if (__syncthreads_or(!ok)) {
@@ -245,9 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
             break;
         }
         pages_waited = i + 1;
-        tc_fence_after();
-        decode_page(sm.stage_k[s], sm.k, tid);
-        decode_page(sm.stage_v[s], sm.v, tid);
+        decode_page<NT>(sm.stage_k[s], sm.k, tid);
+        decode_page<NT>(sm.stage_v[s], sm.v, tid);
         fence_proxy_async_smem();
         __syncthreads();
 
@@ -256,82 +282,80 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
                 issue_page(i + kStages, s);
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = sdesc_sw128(smem_u32(sm.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(smem_u32(sm.k[kk >> 2]) + (kk & 3) * 32, 16, 1024);
-                mma_f16_ss(tmem + kColS, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
-            }
+            for (int r = 0; r < RB; ++r)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = sdesc_sw128(
+                        smem_u32(sm.q[kk >> 2]) + r * 64 * 128 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(smem_u32(sm.k[kk >> 2]) + (kk & 3) * 32, 16, 1024);
+                    mma_f16_ss(tmem + kColS + 64 * r, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                }
             mma_commit(&sm.mma_bar);
         }
+        mma_pending = true;
         ok = mbar_wait(&sm.mma_bar, mma_phase);
-        mma_phase ^= 1u;
+        if (ok) {
+            mma_phase ^= 1u;
+            mma_pending = false;
+        }
         tc_fence_after();
 
-        uint32_t sa[32], sb[32];
-        tmem_ld32(tmem + lane_base + kColS, sa);
-        tmem_ld32(tmem + lane_base + kColS + 32, sb);
-        tmem_ld_wait(sa);
-        tmem_ld_wait(sb);
+        uint32_t sv[32];
+        tmem_ld_16x32bx2_x32(s_addr, sv);
+        tmem_ld_wait(sv);
 
         int n_allow = 0;
-        if (valid) {
+        if (row_valid) {
             const uint32_t word = __ldg(bitrow + (pg >> 5));
             if ((word >> (pg & 31)) & 1u)
                 n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
         }
-        float x[64];
+        const int nh = min(max(n_allow - 32 * hh, 0), 32); // allowed keys in my half
+        float mx = -INFINITY;
+        if (crow >= 0.f) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            x[j] = __uint_as_float(sa[j]) * crow;
-            x[j + 32] = __uint_as_float(sb[j]) * crow;
+            for (int j = 0; j < 32; ++j)
+                if (j < nh)
+                    mx = fmaxf(mx, __uint_as_float(sv[j]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < nh)
+                    mx = fmaxf(mx, -__uint_as_float(sv[j]));
         }
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+        if (n_allow > 0)
+            mx = mx * fabsf(crow);
         float alpha = 1.f;
         bool rescale = false;
-        if (n_allow > 0) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < n_allow)
-                    mx = fmaxf(mx, x[j]);
-            if (mx > m_used + kRescaleLog2) {
-                if (m_used != -INFINITY) {
-                    alpha = ex2(m_used - mx);
-                    rescale = true;
-                    l *= alpha;
-                }
-                m_used = mx;
+        if (n_allow > 0 && mx > m_used + kRescaleLog2) {
+            if (m_used != -INFINITY) {
+                alpha = ex2(m_used - mx);
+                rescale = true;
+                l_part *= alpha;
             }
+            m_used = mx;
         }
-        // P = 2^(x - m) on allowed keys, split into f16 hi + lo, written as the A operand
+        const float negm = n_allow > 0 ? -m_used : 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int j = 8 * c + 2 * e;
-                const float p0 = j < n_allow ? ex2(x[j] - m_used) : 0.f;
-                const float p1 = j + 1 < n_allow ? ex2(x[j + 1] - m_used) : 0.f;
-                l += p0 + p1;
-                const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
-                hi[e] = pack_h2(h0, h1);
-                lo[e] = pack_h2(__float2half_rn(p0 - __half2float(h0)),
-                                __float2half_rn(p1 - __half2float(h1)));
+                const float p0 = j < nh ? ex2(fmaf(__uint_as_float(sv[j]), crow, negm)) : 0.f;
+                const float p1 = j + 1 < nh ? ex2(fmaf(__uint_as_float(sv[j + 1]), crow, negm)) : 0.f;
+                l_part += p0 + p1;
+                split_pair(p0, p1, hi[e], lo[e]);
             }
-            *reinterpret_cast<uint4 *>(sm.p_hi + swz(r, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(sm.p_lo + swz(r, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            const uint32_t o = swz(my_row, 4 * hh + c);
+            *reinterpret_cast<uint4 *>(sm.p_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sm.p_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_base + kColO + 32 * q, o);
-                tmem_ld_wait(o);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                tmem_st32(tmem + lane_base + kColO + 32 * q, o);
-            }
-            tmem_st_wait();
+        if (rescale) {
+            if (hh == 0)
+                sm.alpha[my_row] = alpha;
+            sm.rescale = 1;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -339,14 +363,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
             aborted = true;
             break;
         }
+        if (sm.rescale != 0) {
+            // O^T[d, r] *= alpha[r]: thread = TMEM lane = head dim d (warps of row block 0)
+            if (rb == 0) {
+                tc_fence_after();
+                const uint32_t o_addr = tmem + (static_cast<uint32_t>(32 * qd) << 16) + kColO;
+                for (int c0 = 0; c0 < Npad; c0 += 16) {
+                    uint32_t o[16];
+                    tmem_ld16(o_addr + c0, o);
+                    tmem_ld_wait16(o);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        o[j] = __float_as_uint(__uint_as_float(o[j]) * sm.alpha[c0 + j]);
+                    tmem_st16(o_addr + c0, o);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncthreads(); // every thread has read sm.rescale and alpha by now
+            if (rescale && hh == 0)
+                sm.alpha[my_row] = 1.f;
+            if (tid == 0)
+                sm.rescale = 0;
+        }
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd = sdesc_sw128(smem_u32(sm.v) + kk * 2048, 8192, 1024);
-                mma_f16_ss(tmem + kColO, sdesc_sw128(smem_u32(sm.p_hi) + kk * 32, 16, 1024), bd,
+                const uint64_t ad = sdesc_sw128(smem_u32(sm.v) + kk * 2048, 8192, 1024);
+                mma_f16_ss(tmem + kColO, ad, sdesc_sw128(smem_u32(sm.p_hi) + kk * 32, 16, 1024),
                            kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_f16_ss(tmem + kColO, sdesc_sw128(smem_u32(sm.p_lo) + kk * 32, 16, 1024), bd,
+                mma_f16_ss(tmem + kColO, ad, sdesc_sw128(smem_u32(sm.p_lo) + kk * 32, 16, 1024),
                            kIdescPV, 1u);
             }
             mma_commit(&sm.mma_bar);
@@ -357,9 +404,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
     bool ok = true;
     if (!aborted && mma_pending) {
         ok = mbar_wait(&sm.mma_bar, mma_phase);
-        mma_phase ^= 1u;
-        mma_pending = false;
+        if (ok) {
+            mma_phase ^= 1u;
+            mma_pending = false;
+        }
     }
+    // row sums: combine the two halves, publish 1 / l per row
+    const float l_row = l_part + __shfl_xor_sync(0xFFFFFFFFu, l_part, 16);
+    if (hh == 0)
+        sm.inv_l[my_row] = (row_valid && nU > 0 && l_row > 0.f) ? L.v_scale / l_row : 0.f;
     if (__syncthreads_or(!ok))
         aborted = true;
 
@@ -374,28 +427,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
                 (void)mbar_wait(&sm.mma_bar, mma_phase);
         }
     } else {
-        tc_fence_after();
-        const float inv = (nU > 0 && l > 0.f) ? L.v_scale / l : 0.f;
-        uint16_t *dst = L.O + (static_cast<size_t>(t) * L.Hq + hq) * kHeadDim;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_base + kColO + 32 * q, o);
-            tmem_ld_wait(o);
-            if (valid) {
-                uint32_t pk[16];
+        // O^T (lane d, column r) -> out[r][d] bf16 staged in the (free) k/v tiles, then
+        // written row by row with 16-byte stores.
+        uint16_t *out = reinterpret_cast<uint16_t *>(&sm.k[0][0]);
+        if (rb == 0) {
+            tc_fence_after();
+            const int d = 32 * qd + lane;
+            const uint32_t o_addr = tmem + (static_cast<uint32_t>(32 * qd) << 16) + kColO;
+            for (int c0 = 0; c0 < Npad; c0 += 16) {
+                uint32_t o[16];
+                tmem_ld16(o_addr + c0, o);
+                tmem_ld_wait16(o);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float a = nU > 0 ? __uint_as_float(o[2 * j]) * inv : 0.f;
-                    const float c = nU > 0 ? __uint_as_float(o[2 * j + 1]) * inv : 0.f;
-                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(a, c);
-                    pk[j] = *reinterpret_cast<const uint32_t *>(&v2);
+                    const int r = c0 + j;
+                    if (r < R) {
+                        const float val = nU > 0 ? __uint_as_float(o[j]) * sm.inv_l[r] : 0.f;
+                        out[r * kHeadDim + d] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                    }
                 }
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4 *>(dst + 32 * q + 8 * j) =
-                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
+        }
+        __syncthreads();
+        for (int qn = tid; qn < R * 16; qn += NT) {
+            const int r = qn >> 4, c = qn & 15;
+            uint16_t *dst = L.O + (static_cast<size_t>(sm.row_tok[r]) * L.Hq + sm.row_hq[r]) * kHeadDim;
+            reinterpret_cast<uint4 *>(dst)[c] = reinterpret_cast<const uint4 *>(out + r * kHeadDim)[c];
         }
     }
     tc_fence_before();
@@ -406,19 +463,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn(const AttnLaunch L)
     }
 }
 
+template <int RB>
+cudaError_t launch_rb(const AttnLaunch &L, cudaStream_t st)
+{
+    const size_t smem = sizeof(AttnSmem<RB>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_union_attn<RB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return e;
+    k_union_attn<RB><<<static_cast<unsigned>(L.n_groups), 128 * RB, smem, st>>>(L);
+    return cudaGetLastError();
+}
+
 } // namespace
 
 cudaError_t attn_launch(const AttnLaunch &L, cudaStream_t st)
 {
     if (L.n_groups == 0)
         return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(k_union_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess)
-        return e;
-    const unsigned grid = static_cast<unsigned>(L.n_groups);
-    k_union_attn<<<grid, kThreads, kSmemBytes, st>>>(L);
-    return cudaGetLastError();
+    return L.g * L.G <= 64 ? launch_rb<1>(L, st) : launch_rb<2>(L, st);
 }
 
 } // namespace pw

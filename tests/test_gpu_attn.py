@@ -118,3 +118,41 @@ def test_attn_full_workload_sampled_rows(cfg, W, g):
     ref = oracle.attn_rows(inp, rt, rh)
     got = got.reshape(wl.T, wl.Hq, 128)[rt, rh]
     parity.compare_rows(got, ref, f"{wl.name} W={W} g={g}")
+
+
+@pytest.mark.parametrize("code", [0x01, 0x03, 0x07, 0x87, 0x08])
+def test_subnormal_and_tiny_values_stay_exact(code):
+    # E4M3 subnormals (exponent field 0: m/8 * 2^-6) must survive the decode and the tensor
+    # cores: with every V entry equal to one code, each output row is exactly that value.
+    wl = _small(12, [300], 4, 1, 6)
+    inp = dict(parity.inputs(wl))
+    inp["V_pages"] = np.full_like(inp["V_pages"], code)
+    got, _ = _run(inp, 32, 8)
+    want = oracle.e4m3_to_f64(np.array([code], np.uint8))[0]
+    vals = oracle.bf16_bits_to_f64(got)
+    assert np.all(vals == want), (code, np.unique(vals)[:5], want)
+
+
+def test_subnormal_keys():
+    # Keys made only of subnormal codes: scores are tiny but not zero, and must match.
+    wl = _small(13, [400], 8, 2, 6)
+    inp = dict(parity.inputs(wl))
+    rng = np.random.default_rng(5)
+    K = rng.integers(0, 8, size=inp["K_pages"].shape, dtype=np.uint8)   # codes 0x00..0x07
+    K |= (rng.integers(0, 2, size=K.shape, dtype=np.uint8) << 7)        # random sign
+    inp["K_pages"] = K
+    inp["sm_scale"] = 4000.0    # make the tiny scores matter
+    got, _ = _run(inp, 32, 8)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128), "subnormal K")
+
+
+@pytest.mark.parametrize("scale", [40.0, 400.0])
+def test_frequent_rescales(scale):
+    # A large softmax scale spreads the scores over tens of binades, so the running max of
+    # most rows is raised on many pages and the accumulator rescale runs often.
+    wl = _small(14, [1024, 300], 8, 2, 12, "community", communities=3)
+    inp = dict(parity.inputs(wl))
+    inp["sm_scale"] = inp["sm_scale"] * scale
+    got, _ = _run(inp, 64, 8)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128),
+                        f"scale {scale}")
