@@ -31,16 +31,17 @@
 #include <cuda_runtime.h>
 
 #include "pw_internal.h"
+#include "pw_attn_common.cuh"
 #include "pw_sm100.cuh"
 
 namespace pw {
 namespace {
 
+using namespace attn;
+
 constexpr int kStages = 2;
-constexpr int kPageBytes = kPageTokens * kHeadDim; // one kv head's page, E4M3
-constexpr float kRescaleLog2 = 8.0f;
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
+constexpr int kUnionCache = 512; // union pages whose ids are staged in shared memory
 
 // Operand tiles (rows of 128 bytes = 64 bf16, 16-byte chunks XOR-swizzled by row % 8, 8-row
 // atoms at 1024 bytes):
@@ -61,92 +62,14 @@ struct __align__(1024) AttnSmem {
     float inv_l[RB * 64];
     int32_t row_tok[RB * 64];
     int32_t row_hq[RB * 64];
+    int32_t upage[kUnionCache]; // the group's union pages (logical), first kUnionCache
+    int32_t uphys[kUnionCache]; // and their physical slots
     uint64_t tma_bar[kStages];
     uint64_t mma_bar;
     uint32_t tmem_base;
     int32_t flag;
     int32_t rescale; // some row raised its running max on this page
 };
-
-__device__ __forceinline__ uint32_t swz(int row, int chunk)
-{
-    return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
-{
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// Four E4M3 codes (byte 0 = element 0) -> two bf16x2 words, exactly.  Each byte s.eeee.mmm is
-// widened to a 16-bit half whose high byte repeats the sign (prmt sign mode), shifted so that
-// eeee.mmm lands in the bf16 exponent/mantissa bits 10..4 with the sign at bit 15; that bf16
-// equals the code's value times 2^-120 (subnormal codes included), and one bf16 multiply by
-// 2^120 restores it.
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t &lo, uint32_t &hi)
-{
-    constexpr uint32_t kTwo120 = 0x7B807B80u; // bf16 2^120 in both halves
-    const uint32_t a = (prmt(x, 0u, 0x9180u) << 4) & 0x87F087F0u;
-    const uint32_t b = (prmt(x, 0u, 0xB3A2u) << 4) & 0x87F087F0u;
-    lo = bf16x2_mul(a, kTwo120);
-    hi = bf16x2_mul(b, kTwo120);
-}
-
-// 64 keys x 128 dims E4M3 (row-major) -> two swizzled 64-dim bf16 blocks.  Thread q handles
-// key q/8, dims 16(q%8)..+15 (two 16-byte chunks); threads 4-7 of each quarter-warp store
-// their chunks in the opposite order so a quarter-warp's eight stores hit eight bank groups.
-template <int NT>
-__device__ __forceinline__ void decode_page(const uint8_t *src, uint8_t (*dst)[64 * 128], int tid)
-{
-#pragma unroll
-    for (int rep = 0; rep < 512 / NT; ++rep) {
-        const int q = tid + NT * rep;
-        const int key = q >> 3, c16 = q & 7;
-        const uint4 x = *reinterpret_cast<const uint4 *>(src + key * 128 + c16 * 16);
-        uint4 h0, h1;
-        e4m3x4_to_bf16x4(x.x, h0.x, h0.y);
-        e4m3x4_to_bf16x4(x.y, h0.z, h0.w);
-        e4m3x4_to_bf16x4(x.z, h1.x, h1.y);
-        e4m3x4_to_bf16x4(x.w, h1.z, h1.w);
-        uint8_t *blk = dst[c16 >> 2];
-        const int j0 = (2 * c16) & 7;
-        if (c16 < 4) {
-            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
-            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
-        } else {
-            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
-            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
-        }
-    }
-}
-
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// p -> (hi, lo) bf16 halves of two packed words: hi = p rounded to bf16 (round half up on the
-// bit pattern), lo = p - hi truncated to bf16.
-__device__ __forceinline__ void split_pair(float p0, float p1, uint32_t &hi2, uint32_t &lo2)
-{
-    const uint32_t u0 = __float_as_uint(p0) + 0x8000u;
-    const uint32_t u1 = __float_as_uint(p1) + 0x8000u;
-    const float r0 = p0 - __uint_as_float(u0 & 0xFFFF0000u);
-    const float r1 = p1 - __uint_as_float(u1 & 0xFFFF0000u);
-    hi2 = prmt(u0, u1, 0x7632u);
-    lo2 = prmt(__float_as_uint(r0), __float_as_uint(r1), 0x7632u);
-}
 
 template <int RB>
 __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(const AttnLaunch L)
@@ -198,6 +121,16 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
         sm.row_hq[i] = hq;
         sm.alpha[i] = 1.f;
     }
+    for (int i = tid; i < nU && i < kUnionCache; i += NT) {
+        const int pg = L.union_pages[u0 + i];
+        int phys = L.page_table[static_cast<size_t>(b) * L.max_pages + pg];
+        if (phys < 0 || phys >= L.n_phys) {
+            set_status(L.status, PW_ERR_INVALID_ARG);
+            phys = 0;
+        }
+        sm.upage[i] = pg;
+        sm.uphys[i] = phys;
+    }
     if (tid == 0)
         sm.rescale = 0;
     __syncthreads();
@@ -234,12 +167,19 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
     const uint32_t tmem = sm.tmem_base;
     const uint32_t s_addr = tmem + (static_cast<uint32_t>(32 * qd) << 16) + kColS + 64 * rb;
 
+    auto page_of = [&](int i) -> int {
+        return i < kUnionCache ? sm.upage[i] : L.union_pages[u0 + i];
+    };
     auto issue_page = [&](int i, int s) {
-        const int pg = L.union_pages[u0 + i];
-        int phys = L.page_table[static_cast<size_t>(b) * L.max_pages + pg];
-        if (phys < 0 || phys >= L.n_phys) {
-            set_status(L.status, PW_ERR_INVALID_ARG);
-            phys = 0;
+        int phys;
+        if (i < kUnionCache) {
+            phys = sm.uphys[i];
+        } else {
+            phys = L.page_table[static_cast<size_t>(b) * L.max_pages + L.union_pages[u0 + i]];
+            if (phys < 0 || phys >= L.n_phys) {
+                set_status(L.status, PW_ERR_INVALID_ARG);
+                phys = 0;
+            }
         }
         const size_t off = (static_cast<size_t>(phys) * L.Hkv + h) * kPageBytes;
         mbar_arrive_expect_tx(&sm.tma_bar[s], 2 * kPageBytes);
@@ -257,7 +197,9 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
 
     for (int i = 0; i < nU; ++i) {
         const int s = i % kStages;
-        const int pg = L.union_pages[u0 + i];
+        const int pg = page_of(i);
+        // membership word of my row for this page, fetched now so the decode hides its latency
+        const uint32_t word = row_valid ? __ldg(bitrow + (pg >> 5)) : 0u;
         bool ok = true;
         if (mma_pending) { // previous O^T += V^T P^T: frees v and p, settles O^T
             ok = mbar_wait(&sm.mma_bar, mma_phase);
@@ -278,8 +220,6 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
         __syncthreads();
 
         if (tid == 0) {
-            if (i + kStages < nU)
-                issue_page(i + kStages, s);
             tc_fence_after();
 #pragma unroll
             for (int r = 0; r < RB; ++r)
@@ -291,6 +231,8 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
                     mma_f16_ss(tmem + kColS + 64 * r, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
                 }
             mma_commit(&sm.mma_bar);
+            if (i + kStages < nU) // the stage was consumed by the decode above
+                issue_page(i + kStages, s);
         }
         mma_pending = true;
         ok = mbar_wait(&sm.mma_bar, mma_phase);
@@ -305,11 +247,8 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
         tmem_ld_wait(sv);
 
         int n_allow = 0;
-        if (row_valid) {
-            const uint32_t word = __ldg(bitrow + (pg >> 5));
-            if ((word >> (pg & 31)) & 1u)
-                n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
-        }
+        if ((word >> (pg & 31)) & 1u)
+            n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
         const int nh = min(max(n_allow - 32 * hh, 0), 32); // allowed keys in my half
         float mx = -INFINITY;
         if (crow >= 0.f) {
@@ -337,20 +276,46 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
             m_used = mx;
         }
         const float negm = n_allow > 0 ? -m_used : 0.f;
+        if (__all_sync(0xFFFFFFFFu, nh == 32)) { // whole warp on full pages: no masks
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t hi[4], lo[4];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 8 * c + 2 * e;
-                const float p0 = j < nh ? ex2(fmaf(__uint_as_float(sv[j]), crow, negm)) : 0.f;
-                const float p1 = j + 1 < nh ? ex2(fmaf(__uint_as_float(sv[j + 1]), crow, negm)) : 0.f;
-                l_part += p0 + p1;
-                split_pair(p0, p1, hi[e], lo[e]);
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * c + 2 * e;
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[j]), crow, negm));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[j + 1]), crow, negm));
+                    l_part += p0 + p1;
+                    split_pair(p0, p1, hi[e], lo[e]);
+                }
+                const uint32_t o = swz(my_row, 4 * hh + c);
+                *reinterpret_cast<uint4 *>(sm.p_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm.p_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
-            const uint32_t o = swz(my_row, 4 * hh + c);
-            *reinterpret_cast<uint4 *>(sm.p_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(sm.p_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        } else if (__all_sync(0xFFFFFFFFu, nh == 0)) { // whole warp masked out: P = 0
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t o = swz(my_row, 4 * hh + c);
+                *reinterpret_cast<uint4 *>(sm.p_hi + o) = z;
+                *reinterpret_cast<uint4 *>(sm.p_lo + o) = z;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * c + 2 * e;
+                    const float p0 = j < nh ? ex2(fmaf(__uint_as_float(sv[j]), crow, negm)) : 0.f;
+                    const float p1 = j + 1 < nh ? ex2(fmaf(__uint_as_float(sv[j + 1]), crow, negm)) : 0.f;
+                    l_part += p0 + p1;
+                    split_pair(p0, p1, hi[e], lo[e]);
+                }
+                const uint32_t o = swz(my_row, 4 * hh + c);
+                *reinterpret_cast<uint4 *>(sm.p_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm.p_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
         }
         if (rescale) {
             if (hh == 0)
@@ -482,7 +447,9 @@ cudaError_t attn_launch(const AttnLaunch &L, cudaStream_t st)
 {
     if (L.n_groups == 0)
         return cudaSuccess;
-    return L.g * L.G <= 64 ? launch_rb<1>(L, st) : launch_rb<2>(L, st);
+    // Tiles of up to 64 rows (every g * G <= 64) run on the persistent warp-specialised kernel
+    // (pw_attn_ws.cu); larger tiles on the one-group-per-CTA kernel above.
+    return L.g * L.G <= 64 ? attn_ws_launch(L, st) : launch_rb<2>(L, st);
 }
 
 } // namespace pw

@@ -49,5 +49,6 @@ struct AttnLaunch {
 
 cudaError_t group_launch(const GroupLaunch &L, cudaStream_t st);
 cudaError_t attn_launch(const AttnLaunch &L, cudaStream_t st);
+cudaError_t attn_ws_launch(const AttnLaunch &L, cudaStream_t st); // tiles of <= 64 rows
 
 } // namespace pw
