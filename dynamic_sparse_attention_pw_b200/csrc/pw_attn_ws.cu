@@ -210,57 +210,67 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             }
         }
     } else if (warp == kWarpMma) {
-        // ---------------- MMA issue (one thread) ----------------
-        if (lane == 0) {
-            const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
-            const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // MN-major V^T
-            uint32_t it = 0, nact = 0;
-            bool have_prev = false, ok = true;
-            PendingPV prev{};
-            auto issue_pv = [&](const PendingPV &p) -> bool {
-                const uint32_t pb = p.it & 1u;
-                if (!wait_bar(&sm.p_full[pb], (p.it >> 1) & 1u, &sm.abort_flag) ||
-                    !wait_bar(&sm.v_full[p.vs], (p.it / kNV) & 1u, &sm.abort_flag))
-                    return false;
-                if (p.first && !wait_bar(&sm.o_free[p.ob], ((p.nact >> 1) & 1u) ^ 1u, &sm.abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t idesc = idesc_bf16_f32(128, static_cast<int>(2 * p.npad), true, false);
-                const uint32_t d = tmem + kColO + 128 * p.ob;
-                const uint64_t ad = desc_add(dmn, smem_u32(&sm.v[p.vs][0][0]));
-                const uint64_t bd = desc_add(dsw, smem_u32(sm.p[pb]));
+        // ---------------- MMA issue: the warp runs in lockstep, one elected lane issues ----------------
+        // Lane 0 does the waits and broadcasts the outcome, so every decision is warp-uniform;
+        // operands are computed by the converged warp (uniform registers), the elected lane
+        // (always lane 0) issues the MMAs and their commits.
+        auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            int ok = 1;
+            if (lane == 0)
+                ok = wait_bar(bar, parity, &sm.abort_flag);
+            return __shfl_sync(kFull, ok, 0) != 0;
+        };
+        const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
+        const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // MN-major V^T
+        uint32_t it = 0, nact = 0;
+        bool have_prev = false, ok = true;
+        PendingPV prev{};
+        auto issue_pv = [&](const PendingPV &p) -> bool {
+            const uint32_t pb = p.it & 1u;
+            if (!wwait(&sm.p_full[pb], (p.it >> 1) & 1u) || !wwait(&sm.v_full[p.vs], (p.it / kNV) & 1u))
+                return false;
+            if (p.first && !wwait(&sm.o_free[p.ob], ((p.nact >> 1) & 1u) ^ 1u))
+                return false;
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(128, static_cast<int>(2 * p.npad), true, false);
+            const uint32_t d = tmem + kColO + 128 * p.ob;
+            const uint64_t ad = desc_add(dmn, smem_u32(&sm.v[p.vs][0][0]));
+            const uint64_t bd = desc_add(dsw, smem_u32(sm.p[pb]));
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc,
-                               (p.first && kk == 0) ? 0u : 1u);
+                    mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (p.first && kk == 0) ? 0u : 1u);
                 mma_commit(&sm.v_empty[p.vs]);
                 mma_commit(&sm.o_bar);
-                return true;
-            };
-            for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
-                const int R = L.gsize[gi] * L.G;
-                const uint32_t npad = static_cast<uint32_t>((R + 15) & ~15);
-                const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
-                if (nU == 0)
-                    continue;
-                const uint32_t qb = nact & 1u;
-                if (!wait_bar(&sm.q_full[qb], (nact >> 1) & 1u, &sm.abort_flag)) {
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
+            const int R = L.gsize[gi] * L.G;
+            const uint32_t npad = static_cast<uint32_t>((R + 15) & ~15);
+            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
+            if (nU == 0)
+                continue;
+            const uint32_t qb = nact & 1u;
+            if (!wwait(&sm.q_full[qb], (nact >> 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            const uint64_t aq0 = desc_add(dsw, smem_u32(sm.q[qb][0]));
+            const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][1]));
+            for (int j = 0; j < nU; ++j, ++it) {
+                const uint32_t ks = it % kNK, sb = it & 1u;
+                if (!wwait(&sm.k_full[ks], (it / kNK) & 1u) ||
+                    !wwait(&sm.s_empty[sb], ((it >> 1) & 1u) ^ 1u)) {
                     ok = false;
                     break;
                 }
-                const uint64_t aq0 = desc_add(dsw, smem_u32(sm.q[qb][0]));
-                const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][1]));
-                for (int j = 0; j < nU; ++j, ++it) {
-                    const uint32_t ks = it % kNK, sb = it & 1u;
-                    if (!wait_bar(&sm.k_full[ks], (it / kNK) & 1u, &sm.abort_flag) ||
-                        !wait_bar(&sm.s_empty[sb], ((it >> 1) & 1u) ^ 1u, &sm.abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t bk0 = desc_add(dsw, smem_u32(sm.k[ks][0]));
-                    const uint64_t bk1 = desc_add(dsw, smem_u32(sm.k[ks][1]));
-                    const uint32_t ds = tmem + 64 * sb;
+                tc_fence_after();
+                const uint64_t bk0 = desc_add(dsw, smem_u32(sm.k[ks][0]));
+                const uint64_t bk1 = desc_add(dsw, smem_u32(sm.k[ks][1]));
+                const uint32_t ds = tmem + 64 * sb;
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16_ss(ds, aq0 + 2u * kk, bk0 + 2u * kk, kIdescS, kk > 0 ? 1u : 0u);
@@ -271,18 +281,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     mma_commit(&sm.k_empty[ks]);
                     if (j == nU - 1)
                         mma_commit(&sm.q_empty[qb]);
-                    if (have_prev && !issue_pv(prev)) {
-                        ok = false;
-                        break;
-                    }
-                    prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0};
-                    have_prev = true;
                 }
-                ++nact;
+                __syncwarp();
+                if (have_prev && !issue_pv(prev)) {
+                    ok = false;
+                    break;
+                }
+                prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0};
+                have_prev = true;
             }
-            if (ok && have_prev)
-                (void)issue_pv(prev);
+            ++nact;
         }
+        if (ok && have_prev)
+            (void)issue_pv(prev);
     } else if (warp < kWarpSm0) {
         // ---------------- decode: Q tiles and E4M3 -> bf16 K/V tiles (256 threads) ----------------
         uint32_t it = 0, nact = 0;
@@ -344,6 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         const float crow = L.sm_scale * L.k_scale * kLog2e;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
         uint32_t it = 0, nact = 0;
+        // Products (one o_bar phase per page) known complete: [0, pv_done).  A parity wait is
+        // only unambiguous one phase ahead of what is known complete, so wait_pv steps through
+        // the phases in order.  Seeing S of page i also proves the product of page i-2 complete
+        // (S_i is issued after it).
+        uint32_t pv_done = 0;
+        auto wait_pv = [&](uint32_t x) -> bool { // product of page x complete
+            for (; pv_done <= x; ++pv_done)
+                if (!wait_bar(&sm.o_bar, pv_done & 1u, &sm.abort_flag))
+                    return false;
+            return true;
+        };
         bool ok = true;
         for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
             const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
@@ -397,6 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     ok = false;
                     break;
                 }
+                if (it >= 2 && pv_done < it - 1)
+                    pv_done = it - 1;
                 tc_fence_after();
                 uint32_t sv[32];
                 tmem_ld_16x32bx2_x32(tmem + lane_base + 64 * sb, sv);
@@ -492,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     // O^T[d, r] *= alpha[r] for both accumulator halves, after the previous
                     // page's product (the only one that may still run: S of this page, issued
                     // after the products before it, is complete).
-                    ok = j == 0 || wait_bar(&sm.o_bar, (it - 1) & 1u, &sm.abort_flag);
+                    ok = j == 0 || wait_pv(it - 1);
                     if (softmax_bar_or(!ok)) {
                         ok = false;
                         break;
@@ -516,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             if (!ok)
                 break;
             // epilogue: the group's last product is page it - 1
-            ok = wait_bar(&sm.o_bar, (it - 1) & 1u, &sm.abort_flag);
+            ok = wait_pv(it - 1);
             const float l_row = l_part + __shfl_xor_sync(kFull, l_part, 16);
             if (hh == 0)
                 sm.inv_l[row] = (valid && l_row > 0.f) ? L.v_scale / l_row : 0.f;
@@ -565,9 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 (void)mbar_wait(&sm.full_stage[s], (last / kNS) & 1u);
             }
         }
-        if (warp == kWarpMma && lane == 0) {
-            mma_commit(&sm.drain_bar);
-            (void)mbar_wait(&sm.drain_bar, 0);
+        if (warp == kWarpMma) {
+            if (elect_one()) {
+                mma_commit(&sm.drain_bar);
+                (void)mbar_wait(&sm.drain_bar, 0);
+            }
+            __syncwarp();
         }
     }
     __syncthreads();

@@ -127,32 +127,16 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint
                  : "memory");
 }
 
-// Same MMA issued from a converged warp: every lane executes this with identical operands and
-// lane 0 (the lane that also commits) issues it.  Issuing from a converged warp keeps the
-// operands warp-uniform, which roughly halves the issue cost per instruction compared with a
-// single divergent thread.
-__device__ __forceinline__ void mma_f16_ss_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                uint32_t idesc, uint32_t accumulate)
+// One lane of a converged warp: elect.sync picks the lowest active lane, so a warp that stays
+// converged always elects the same lane (the one whose MMAs a later commit tracks).
+__device__ __forceinline__ bool elect_one()
 {
-    asm volatile("{\n\t.reg .pred p, e;\n\t"
-                 ".reg .u32 l;\n\t"
-                 "setp.ne.b32 p, %4, 0;\n\t"
-                 "mov.u32 l, %%laneid;\n\t"
-                 "setp.eq.u32 e, l, 0;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-                 : "memory");
-}
-
-// Commit from a converged warp, by lane 0 (the lane that issued the MMAs).
-__device__ __forceinline__ void mma_commit_warp(uint64_t *bar)
-{
-    asm volatile("{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
-                 "mov.u32 l, %%laneid;\n\t"
-                 "setp.eq.u32 e, l, 0;\n\t"
-                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
+    uint32_t e;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "elect.sync _|p, 0xffffffff;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}\n"
+                 : "=r"(e));
+    return e != 0;
 }
 
 // Arrive once on `bar` when every tcgen05.mma this thread issued so far has completed.
