@@ -8,9 +8,10 @@
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
 //   warps 0-7    decode   Q tile of each group (bf16, gathered by query ID); E4M3 K and V
 //                         pages -> bf16 operand tiles
-//   warps 8-11   softmax  S -> P for each page, lazy O^T rescale, epilogue of each group
-//   warp 12      load     bulk copies (TMA) of the union pages into a 3-stage FP8 ring
-//   warp 13      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
+//   warps 8-15   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
+//                         O^T rescale, epilogue of each group
+//   warp 16      load     bulk copies (TMA) of the union pages into a 3-stage FP8 ring
+//   warp 17      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
 // (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, which the
 // epilogue adds.  K and V have separate buffers: a K slot is free once S is done, a V slot
@@ -32,9 +33,11 @@ using namespace attn;
 constexpr int kNS = 3;        // FP8 page stages
 constexpr int kNK = 2;        // bf16 K slots
 constexpr int kNV = 3;        // bf16 V slots
+static_assert(kNK == 2, "s_done doubles as the K-slot release: it needs as many K slots as S buffers");
 constexpr int kDecThreads = 256;
-constexpr int kWarpSm0 = 8, kWarpLoad = 12, kWarpMma = 13;
-constexpr int kThreads = 448; // 14 warps
+constexpr int kSmThreads = 256;
+constexpr int kWarpSm0 = 8, kWarpLoad = 16, kWarpMma = 17;
+constexpr int kThreads = 576; // 18 warps
 constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 64, O^T[0..1] at 128 / 256
 constexpr uint32_t kColO = 128;
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
@@ -50,14 +53,15 @@ struct __align__(1024) WsSmem {
     uint16_t out[64 * 128];      // epilogue staging, bf16 [row][head dim]
     float alpha[2][64];
     float inv_l[64];
+    float qmax[64][4]; // per-row partial maxima / sums exchanged by the row's four threads
     int32_t row_tok[64];
     int32_t row_hq[64];
     uint64_t full_stage[kNS], empty_stage[kNS];
-    uint64_t k_full[kNK], k_empty[kNK];
-    uint64_t v_full[kNV], v_empty[kNV];
-    uint64_t s_full[2], s_empty[2];
+    uint64_t k_full[kNK];
+    uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
+    uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete (and its K slot free)
+    uint64_t s_empty[2];
     uint64_t p_full[2];
-    uint64_t o_bar;
     uint64_t q_full[2], q_empty[2];
     uint64_t o_free[2];
     uint64_t drain_bar;
@@ -89,13 +93,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
     return true;
 }
 
-// Named barrier 1 over the 128 softmax threads, returning whether any of them passed `pred`.
+// Named barrier 1 over the 256 softmax threads, returning whether any of them passed `pred`.
 __device__ __forceinline__ bool softmax_bar_or(bool pred)
 {
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\t"
                  "setp.ne.u32 q, %1, 0;\n\t"
-                 "bar.red.or.pred p, 1, 128, q;\n\t"
+                 "bar.red.or.pred p, 1, 256, q;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}\n"
                  : "=r"(r)
                  : "r"(pred ? 1u : 0u)
@@ -105,7 +109,7 @@ __device__ __forceinline__ bool softmax_bar_or(bool pred)
 
 __device__ __forceinline__ void softmax_bar()
 {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 // A descriptor's start-address field is (address >> 4) in its low 14 bits: a descriptor for
@@ -113,6 +117,25 @@ __device__ __forceinline__ void softmax_bar()
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t off_bytes)
 {
     return d + static_cast<uint64_t>(off_bytes >> 4);
+}
+
+// One arrival per warp: every lane's prior writes are ordered before lane 0's arrive.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane)
+{
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(bar);
+}
+
+// Lane 0 waits; the warp follows (lane 0's acquire is passed on by the warp barrier).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *abort_flag, int lane)
+{
+    int ok = 1;
+    if (lane == 0)
+        ok = wait_bar(bar, parity, abort_flag);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok != 0;
 }
 
 struct PendingPV {
@@ -134,27 +157,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         return;
 
     if (tid == 0) {
+        // Arrivals from the decode and softmax roles are one per warp (after __syncwarp).
         for (int s = 0; s < kNS; ++s) {
             mbar_init(&sm.full_stage[s], 1);
-            mbar_init(&sm.empty_stage[s], kDecThreads);
+            mbar_init(&sm.empty_stage[s], kDecThreads / 32);
         }
-        for (int s = 0; s < kNK; ++s) {
-            mbar_init(&sm.k_full[s], kDecThreads);
-            mbar_init(&sm.k_empty[s], 1);
-        }
+        for (int s = 0; s < kNK; ++s)
+            mbar_init(&sm.k_full[s], kDecThreads / 32);
         for (int s = 0; s < kNV; ++s) {
-            mbar_init(&sm.v_full[s], kDecThreads);
+            mbar_init(&sm.v_full[s], kDecThreads / 32);
             mbar_init(&sm.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.s_full[s], 1);
-            mbar_init(&sm.s_empty[s], 128);
-            mbar_init(&sm.p_full[s], 128);
-            mbar_init(&sm.q_full[s], kDecThreads);
+            mbar_init(&sm.s_done[s], 1);
+            mbar_init(&sm.s_empty[s], kSmThreads / 32);
+            mbar_init(&sm.p_full[s], kSmThreads / 32);
+            mbar_init(&sm.q_full[s], kDecThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
-            mbar_init(&sm.o_free[s], 128);
+            mbar_init(&sm.o_free[s], kSmThreads / 32);
         }
-        mbar_init(&sm.o_bar, 1);
         mbar_init(&sm.drain_bar, 1);
         sm.abort_flag = 0;
         sm.load_issued = 0;
@@ -241,7 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (p.first && kk == 0) ? 0u : 1u);
                 mma_commit(&sm.v_empty[p.vs]);
-                mma_commit(&sm.o_bar);
             }
             __syncwarp();
             return true;
@@ -277,8 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16_ss(ds, aq1 + 2u * kk, bk1 + 2u * kk, kIdescS, 1u);
-                    mma_commit(&sm.s_full[sb]);
-                    mma_commit(&sm.k_empty[ks]);
+                    mma_commit(&sm.s_done[sb]); // kNK == 2: the K slot index is sb too
                     if (j == nU - 1)
                         mma_commit(&sm.q_empty[qb]);
                 }
@@ -305,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             if (nU == 0)
                 continue;
             const uint32_t qb = nact & 1u;
-            if (!wait_bar(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag)) {
+            if (!warp_wait(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag, lane)) {
                 ok = false;
                 break;
             }
@@ -324,45 +343,60 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 *reinterpret_cast<uint4 *>(sm.q[qb][c >> 3] + swz(row, c & 7)) = val;
             }
             fence_proxy_async_smem();
-            mbar_arrive(&sm.q_full[qb]);
+            warp_arrive(&sm.q_full[qb], lane);
             for (int j = 0; j < nU; ++j, ++it) {
                 const uint32_t st = it % kNS, ks = it % kNK, vs = it % kNV;
-                if (!wait_bar(&sm.full_stage[st], (it / kNS) & 1u, &sm.abort_flag) ||
-                    !wait_bar(&sm.k_empty[ks], ((it / kNK) & 1u) ^ 1u, &sm.abort_flag)) {
+                if (!warp_wait(&sm.full_stage[st], (it / kNS) & 1u, &sm.abort_flag, lane) ||
+                    !warp_wait(&sm.s_done[ks], ((it / kNK) & 1u) ^ 1u, &sm.abort_flag, lane)) {
                     ok = false;
                     break;
                 }
                 decode_page<kDecThreads>(sm.stage_k[st], sm.k[ks], tid);
                 fence_proxy_async_smem();
-                mbar_arrive(&sm.k_full[ks]);
-                if (!wait_bar(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag)) {
+                warp_arrive(&sm.k_full[ks], lane);
+                if (!warp_wait(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag, lane)) {
                     ok = false;
                     break;
                 }
                 decode_page<kDecThreads>(sm.stage_v[st], sm.v[vs], tid);
                 fence_proxy_async_smem();
-                mbar_arrive(&sm.v_full[vs]);
-                mbar_arrive(&sm.empty_stage[st]);
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.v_full[vs]);
+                    mbar_arrive(&sm.empty_stage[st]);
+                }
             }
             ++nact;
         }
     } else {
-        // ---------------- softmax + epilogue (128 threads, warps 8-11) ----------------
-        const int st = tid - kWarpSm0 * 32; // 0..127, also the TMEM lane (head dim) in the epilogue
-        const int qd = warp - kWarpSm0;     // TMEM lane quadrant
+        // ---------------- softmax + epilogue (256 threads, warps 8-15) ----------------
+        // Four threads share a row: warp (quadrant qd, half hw) reads TMEM lanes of rows
+        // 16 qd .. 16 qd + 15 and keys 32 hw .. 32 hw + 31; lane / 16 picks 16 of those keys.
+        // A row's running max m is identical in its four threads and changes only on the slow
+        // path, which runs when some element of some row exceeds its m by more than 2^8 (one
+        // OR over all 256 threads decides), so the common path needs no exchange.
+        const int st = tid - kWarpSm0 * 32; // 0..255
+        const int sw = warp - kWarpSm0;     // 0..7
+        const int qd = sw & 3;              // TMEM lane quadrant
+        const int hw = sw >> 2;             // key half of the page read by this warp
         const int row = 16 * qd + (lane & 15);
-        const int hh = lane >> 4;
+        const int qq = 2 * hw + (lane >> 4); // 16-key quarter of the page owned by this thread
+        const int dlane = 32 * qd + lane;    // TMEM lane = head dimension, in the epilogue
         const float crow = L.sm_scale * L.k_scale * kLog2e;
+        const float acrow = fabsf(crow);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
         uint32_t it = 0, nact = 0;
-        // Products (one o_bar phase per page) known complete: [0, pv_done).  A parity wait is
+        // Products known complete: [0, pv_done).  A parity wait is
         // only unambiguous one phase ahead of what is known complete, so wait_pv steps through
         // the phases in order.  Seeing S of page i also proves the product of page i-2 complete
         // (S_i is issued after it).
+        // v_empty[x % kNV] completes once per product of page x; waited in page order it is
+        // unambiguous.  Lane 0 of each warp waits; the collective check that follows every
+        // call synchronises the rest.
         uint32_t pv_done = 0;
         auto wait_pv = [&](uint32_t x) -> bool { // product of page x complete
             for (; pv_done <= x; ++pv_done)
-                if (!wait_bar(&sm.o_bar, pv_done & 1u, &sm.abort_flag))
+                if (lane == 0 && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
                     return false;
             return true;
         };
@@ -384,16 +418,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 own = pos >> 6;
                 bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
             }
-            if (hh == 0) {
+            if (qq == 0) {
                 sm.row_tok[row] = static_cast<int32_t>(tok);
                 sm.row_hq[row] = hq;
             }
             if (nU == 0) {
                 if (valid) { // no union page: every row of the group is empty
                     uint4 *dst = reinterpret_cast<uint4 *>(
-                        L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim + 64 * hh);
+                        L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim + 32 * qq);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
+                    for (int c = 0; c < 4; ++c)
                         dst[c] = make_uint4(0u, 0u, 0u, 0u);
                 }
                 softmax_bar();
@@ -414,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 const uint32_t sb = it & 1u, pb = it & 1u;
                 // every abort decision of this role is collective: a thread that left alone
                 // would strand the others at the named barrier or in a warp-wide TMEM load
-                ok = wait_bar(&sm.s_full[sb], (it >> 1) & 1u, &sm.abort_flag);
+                ok = lane != 0 || wait_bar(&sm.s_done[sb], (it >> 1) & 1u, &sm.abort_flag);
                 if (softmax_bar_or(!ok)) {
                     ok = false;
                     break;
@@ -422,134 +456,123 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 if (it >= 2 && pv_done < it - 1)
                     pv_done = it - 1;
                 tc_fence_after();
-                uint32_t sv[32];
-                tmem_ld_16x32bx2_x32(tmem + lane_base + 64 * sb, sv);
-                tmem_ld_wait(sv);
+                uint32_t sv[16];
+                tmem_ld_16x32bx2_x16(tmem + lane_base + 64 * sb + 32 * hw, sv);
+                tmem_ld_wait16(sv);
                 tc_fence_before();
-                mbar_arrive(&sm.s_empty[sb]);
+                warp_arrive(&sm.s_empty[sb], lane);
 
                 int n_allow = 0;
                 if ((word >> (pg & 31)) & 1u)
                     n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
-                const int nh = min(max(n_allow - 32 * hh, 0), 32);
-                float mx = -INFINITY;
+                const int nq = min(max(n_allow - 16 * qq, 0), 16); // allowed keys in my quarter
+                float lm = -INFINITY;
                 if (crow >= 0.f) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (e < nh)
-                            mx = fmaxf(mx, __uint_as_float(sv[e]));
+                    for (int e = 0; e < 16; ++e)
+                        if (e < nq)
+                            lm = fmaxf(lm, __uint_as_float(sv[e]));
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (e < nh)
-                            mx = fmaxf(mx, -__uint_as_float(sv[e]));
+                    for (int e = 0; e < 16; ++e)
+                        if (e < nq)
+                            lm = fmaxf(lm, -__uint_as_float(sv[e]));
                 }
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                if (n_allow > 0)
-                    mx = mx * fabsf(crow);
-                float alpha = 1.f;
-                bool rescale = false;
-                if (n_allow > 0 && mx > m_used + kRescaleLog2) {
-                    if (m_used != -INFINITY) {
-                        alpha = ex2(m_used - mx);
-                        rescale = true;
-                        l_part *= alpha;
+                if (nq > 0)
+                    lm *= acrow;
+                if (softmax_bar_or(nq > 0 && lm > m_used + kRescaleLog2)) {
+                    // slow path: the row's four threads agree on its max
+                    sm.qmax[row][qq] = lm;
+                    softmax_bar();
+                    const float M = fmaxf(fmaxf(sm.qmax[row][0], sm.qmax[row][1]),
+                                          fmaxf(sm.qmax[row][2], sm.qmax[row][3]));
+                    float alpha = 1.f;
+                    bool rescale = false;
+                    if (M > m_used + kRescaleLog2) {
+                        if (m_used != -INFINITY) {
+                            alpha = ex2(m_used - M);
+                            rescale = true;
+                            l_part *= alpha;
+                        }
+                        m_used = M;
                     }
-                    m_used = mx;
+                    if (qq == 0)
+                        sm.alpha[pb][row] = rescale ? alpha : 1.f;
+                    if (softmax_bar_or(rescale)) {
+                        // O^T[d, r] *= alpha[r] for both accumulator halves, after the previous
+                        // page's product (the only one that may still run).
+                        ok = j == 0 || wait_pv(it - 1);
+                        if (softmax_bar_or(!ok)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        for (int c0 = 16 * hw; c0 < 2 * npad; c0 += 32) {
+                            uint32_t o[16];
+                            tmem_ld16(o_addr + c0, o);
+                            tmem_ld_wait16(o);
+                            const int r0 = c0 < npad ? c0 : c0 - npad;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[pb][r0 + e]);
+                            tmem_st16(o_addr + c0, o);
+                        }
+                        tmem_st_wait();
+                    }
                 }
-                const float negm = n_allow > 0 ? -m_used : 0.f;
+                const float negm = m_used == -INFINITY ? 0.f : -m_used;
                 // P buffer pb was last read by the product of page it-2, complete since
-                // S of page it (issued after it) is.
-                // Rows 0..npad-1 hold P_hi, rows npad..2 npad-1 P_lo; only rows < npad write.
+                // S of page it (issued after it) is.  Rows 0..npad-1 hold P_hi, rows
+                // npad..2 npad-1 P_lo; only rows < npad write.
                 uint8_t *phi = sm.p[pb], *plo = sm.p[pb] + npad * 128;
-                if (__all_sync(kFull, nh == 32)) {
+                uint32_t hi[8], lo[8];
+                if (__all_sync(kFull, nq == 16)) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t hi[4], lo[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int x = 8 * c + 2 * e;
-                            const float p0 = ex2(fmaf(__uint_as_float(sv[x]), crow, negm));
-                            const float p1 = ex2(fmaf(__uint_as_float(sv[x + 1]), crow, negm));
-                            l_part += p0 + p1;
-                            split_pair(p0, p1, hi[e], lo[e]);
-                        }
-                        const uint32_t o = swz(row, 4 * hh + c);
-                        if (row < npad) {
-                            *reinterpret_cast<uint4 *>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                            *reinterpret_cast<uint4 *>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        }
-                    }
-                } else if (__all_sync(kFull, nh == 0)) {
-                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t o = swz(row, 4 * hh + c);
-                        if (row < npad) {
-                            *reinterpret_cast<uint4 *>(phi + o) = z;
-                            *reinterpret_cast<uint4 *>(plo + o) = z;
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), crow, negm));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow, negm));
+                        l_part += p0 + p1;
+                        split_pair(p0, p1, hi[e], lo[e]);
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t hi[4], lo[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int x = 8 * c + 2 * e;
-                            const float p0 = x < nh ? ex2(fmaf(__uint_as_float(sv[x]), crow, negm)) : 0.f;
-                            const float p1 = x + 1 < nh ? ex2(fmaf(__uint_as_float(sv[x + 1]), crow, negm)) : 0.f;
-                            l_part += p0 + p1;
-                            split_pair(p0, p1, hi[e], lo[e]);
-                        }
-                        const uint32_t o = swz(row, 4 * hh + c);
-                        if (row < npad) {
-                            *reinterpret_cast<uint4 *>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                            *reinterpret_cast<uint4 *>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), crow, negm)) : 0.f;
+                        const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow, negm)) : 0.f;
+                        l_part += p0 + p1;
+                        split_pair(p0, p1, hi[e], lo[e]);
                     }
                 }
-                if (hh == 0)
-                    sm.alpha[pb][row] = rescale ? alpha : 1.f;
+                if (row < npad) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t o = swz(row, 2 * qq + c);
+                        *reinterpret_cast<uint4 *>(phi + o) =
+                            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                        *reinterpret_cast<uint4 *>(plo + o) =
+                            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                    }
+                }
                 fence_proxy_async_smem();
-                if (softmax_bar_or(rescale)) {
-                    // O^T[d, r] *= alpha[r] for both accumulator halves, after the previous
-                    // page's product (the only one that may still run: S of this page, issued
-                    // after the products before it, is complete).
-                    ok = j == 0 || wait_pv(it - 1);
-                    if (softmax_bar_or(!ok)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    for (int c0 = 0; c0 < 2 * npad; c0 += 16) {
-                        uint32_t o[16];
-                        tmem_ld16(o_addr + c0, o);
-                        tmem_ld_wait16(o);
-                        const int r0 = c0 < npad ? c0 : c0 - npad;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[pb][r0 + e]);
-                        tmem_st16(o_addr + c0, o);
-                    }
-                    tmem_st_wait();
-                }
                 tc_fence_before();
-                mbar_arrive(&sm.p_full[pb]);
+                warp_arrive(&sm.p_full[pb], lane);
             }
             if (!ok)
                 break;
             // epilogue: the group's last product is page it - 1
             ok = wait_pv(it - 1);
-            const float l_row = l_part + __shfl_xor_sync(kFull, l_part, 16);
-            if (hh == 0)
-                sm.inv_l[row] = (valid && l_row > 0.f) ? L.v_scale / l_row : 0.f;
+            sm.qmax[row][qq] = l_part;
             if (softmax_bar_or(!ok)) {
                 ok = false;
                 break;
             }
+            if (qq == 0) {
+                const float l_row = sm.qmax[row][0] + sm.qmax[row][1] + sm.qmax[row][2] + sm.qmax[row][3];
+                sm.inv_l[row] = (valid && l_row > 0.f) ? L.v_scale / l_row : 0.f;
+            }
+            softmax_bar();
             tc_fence_after();
-            for (int c0 = 0; c0 < npad; c0 += 16) {
+            for (int c0 = 16 * hw; c0 < npad; c0 += 32) {
                 uint32_t ohi[16], olo[16];
                 tmem_ld16(o_addr + c0, ohi);
                 tmem_ld16(o_addr + npad + c0, olo);
@@ -559,19 +582,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 for (int e = 0; e < 16; ++e) {
                     const int r = c0 + e;
                     const float val = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * sm.inv_l[r];
-                    sm.out[r * kHeadDim + st] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                    sm.out[r * kHeadDim + dlane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
                 }
             }
             tc_fence_before();
-            mbar_arrive(&sm.o_free[ob]);
+            warp_arrive(&sm.o_free[ob], lane);
             softmax_bar();
-            for (int qn = st; qn < R * 16; qn += 128) {
+            for (int qn = st; qn < R * 16; qn += kSmThreads) {
                 const int r = qn >> 4, c = qn & 15;
                 uint16_t *dst = L.O + (static_cast<size_t>(sm.row_tok[r]) * L.Hq + sm.row_hq[r]) * kHeadDim;
                 reinterpret_cast<uint4 *>(dst)[c] =
                     reinterpret_cast<const uint4 *>(sm.out + r * kHeadDim)[c];
             }
-            softmax_bar(); // row_tok, inv_l and out are rewritten by the next group
+            softmax_bar(); // row_tok, qmax, inv_l and out are rewritten by the next group
             ++nact;
         }
     }
