@@ -9,14 +9,17 @@
 //   warps 0-7    decode   Q tile of each group (bf16, gathered by query ID); E4M3 K and V
 //                         pages -> bf16 operand tiles
 //   warps 8-15   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
-//                         O^T rescale, epilogue of each group
-//   warp 16      load     bulk copies (TMA) of the union pages into a 3-stage FP8 ring
-//   warp 17      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
+//                         O^T rescale, per-row sums of each group
+//   warps 16-19  epilogue O^T of a finished group -> bf16 rows of O (one warp per TMEM lane
+//                         quadrant), while the softmax warps already work on the next group
+//   warp 20      load     bulk copies (TMA) of the union pages into a 3-stage FP8 ring
+//   warp 21      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
 // (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, which the
 // epilogue adds.  K and V have separate buffers: a K slot is free once S is done, a V slot
-// once the product is done.  Every hand-off is an mbarrier; every wait is bounded and, when it
-// runs out, sets an abort flag that releases the other roles.
+// once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
+// mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
+// other roles.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,13 +34,14 @@ namespace {
 using namespace attn;
 
 constexpr int kNS = 3;        // FP8 page stages
-constexpr int kNK = 2;        // bf16 K slots
+constexpr int kNK = 3;        // bf16 K slots
 constexpr int kNV = 3;        // bf16 V slots
-static_assert(kNK == 2, "s_done doubles as the K-slot release: it needs as many K slots as S buffers");
 constexpr int kDecThreads = 256;
 constexpr int kSmThreads = 256;
-constexpr int kWarpSm0 = 8, kWarpLoad = 16, kWarpMma = 17;
-constexpr int kThreads = 576; // 18 warps
+constexpr int kEpiThreads = 128;
+constexpr int kWarpSm0 = 8, kWarpEpi0 = 16, kWarpLoad = 20, kWarpMma = 21;
+constexpr int kThreads = 704; // 22 warps
+static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
 constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 64, O^T[0..1] at 128 / 256
 constexpr uint32_t kColO = 128;
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
@@ -50,20 +54,19 @@ struct __align__(1024) WsSmem {
     uint8_t p[2][128 * 128];     // [buffer][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
     uint8_t stage_k[kNS][kPageBytes];
     uint8_t stage_v[kNS][kPageBytes];
-    uint16_t out[64 * 128];      // epilogue staging, bf16 [row][head dim]
     float alpha[2][64];
-    float inv_l[64];
-    float qmax[64][4]; // per-row partial maxima / sums exchanged by the row's four threads
-    int32_t row_tok[64];
-    int32_t row_hq[64];
+    float qmax[64][4];    // per-row partial maxima exchanged by the row's four threads
+    float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
     uint64_t full_stage[kNS], empty_stage[kNS];
-    uint64_t k_full[kNK];
+    uint64_t k_full[kNK], k_empty[kNK];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
-    uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete (and its K slot free)
+    uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete
     uint64_t s_empty[2];
     uint64_t p_full[2];
     uint64_t q_full[2], q_empty[2];
-    uint64_t o_free[2];
+    uint64_t o_full[2]; // last product of the group in O buffer b complete
+    uint64_t l_full[2]; // row sums of that group published
+    uint64_t o_free[2]; // epilogue done with O buffer b (and lsum[b])
     uint64_t drain_bar;
     uint32_t load_issued; // pages whose copies the load warp issued (for the abort drain)
     uint32_t tmem_base;
@@ -140,7 +143,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_
 
 struct PendingPV {
     uint32_t it, vs, ob, nact, npad;
-    bool first;
+    bool first, last;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch L)
@@ -162,8 +165,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             mbar_init(&sm.full_stage[s], 1);
             mbar_init(&sm.empty_stage[s], kDecThreads / 32);
         }
-        for (int s = 0; s < kNK; ++s)
+        for (int s = 0; s < kNK; ++s) {
             mbar_init(&sm.k_full[s], kDecThreads / 32);
+            mbar_init(&sm.k_empty[s], 1);
+        }
         for (int s = 0; s < kNV; ++s) {
             mbar_init(&sm.v_full[s], kDecThreads / 32);
             mbar_init(&sm.v_empty[s], 1);
@@ -174,7 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             mbar_init(&sm.p_full[s], kSmThreads / 32);
             mbar_init(&sm.q_full[s], kDecThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
-            mbar_init(&sm.o_free[s], kSmThreads / 32);
+            mbar_init(&sm.o_full[s], 1);
+            mbar_init(&sm.l_full[s], kSmThreads / 32);
+            mbar_init(&sm.o_free[s], kEpiThreads / 32);
         }
         mbar_init(&sm.drain_bar, 1);
         sm.abort_flag = 0;
@@ -262,6 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 for (int kk = 0; kk < 4; ++kk)
                     mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (p.first && kk == 0) ? 0u : 1u);
                 mma_commit(&sm.v_empty[p.vs]);
+                if (p.last)
+                    mma_commit(&sm.o_full[p.ob]);
             }
             __syncwarp();
             return true;
@@ -297,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f16_ss(ds, aq1 + 2u * kk, bk1 + 2u * kk, kIdescS, 1u);
-                    mma_commit(&sm.s_done[sb]); // kNK == 2: the K slot index is sb too
+                    mma_commit(&sm.s_done[sb]);
+                    mma_commit(&sm.k_empty[ks]);
                     if (j == nU - 1)
                         mma_commit(&sm.q_empty[qb]);
                 }
@@ -306,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     ok = false;
                     break;
                 }
-                prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0};
+                prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0, j == nU - 1};
                 have_prev = true;
             }
             ++nact;
@@ -347,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             for (int j = 0; j < nU; ++j, ++it) {
                 const uint32_t st = it % kNS, ks = it % kNK, vs = it % kNV;
                 if (!warp_wait(&sm.full_stage[st], (it / kNS) & 1u, &sm.abort_flag, lane) ||
-                    !warp_wait(&sm.s_done[ks], ((it / kNK) & 1u) ^ 1u, &sm.abort_flag, lane)) {
+                    !warp_wait(&sm.k_empty[ks], ((it / kNK) & 1u) ^ 1u, &sm.abort_flag, lane)) {
                     ok = false;
                     break;
                 }
@@ -368,20 +378,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             }
             ++nact;
         }
-    } else {
-        // ---------------- softmax + epilogue (256 threads, warps 8-15) ----------------
+    } else if (warp < kWarpEpi0) {
+        // ---------------- softmax (256 threads, warps 8-15) ----------------
         // Four threads share a row: warp (quadrant qd, half hw) reads TMEM lanes of rows
         // 16 qd .. 16 qd + 15 and keys 32 hw .. 32 hw + 31; lane / 16 picks 16 of those keys.
         // A row's running max m is identical in its four threads and changes only on the slow
         // path, which runs when some element of some row exceeds its m by more than 2^8 (one
         // OR over all 256 threads decides), so the common path needs no exchange.
-        const int st = tid - kWarpSm0 * 32; // 0..255
         const int sw = warp - kWarpSm0;     // 0..7
         const int qd = sw & 3;              // TMEM lane quadrant
         const int hw = sw >> 2;             // key half of the page read by this warp
         const int row = 16 * qd + (lane & 15);
         const int qq = 2 * hw + (lane >> 4); // 16-key quarter of the page owned by this thread
-        const int dlane = 32 * qd + lane;    // TMEM lane = head dimension, in the epilogue
         const float crow = L.sm_scale * L.k_scale * kLog2e;
         const float acrow = fabsf(crow);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
@@ -418,10 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 own = pos >> 6;
                 bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
             }
-            if (qq == 0) {
-                sm.row_tok[row] = static_cast<int32_t>(tok);
-                sm.row_hq[row] = hq;
-            }
             if (nU == 0) {
                 if (valid) { // no union page: every row of the group is empty
                     uint4 *dst = reinterpret_cast<uint4 *>(
@@ -430,7 +434,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     for (int c = 0; c < 4; ++c)
                         dst[c] = make_uint4(0u, 0u, 0u, 0u);
                 }
-                softmax_bar();
                 continue;
             }
             const uint32_t ob = nact & 1u;
@@ -559,42 +562,74 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             }
             if (!ok)
                 break;
-            // epilogue: the group's last product is page it - 1
-            ok = wait_pv(it - 1);
-            sm.qmax[row][qq] = l_part;
+            // Publish the row-sum partials of this group for the epilogue warps.  lsum[ob] was
+            // last read by the epilogue of group nact - 2, which released it with o_free[ob].
+            ok = lane != 0 || wait_bar(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
             if (softmax_bar_or(!ok)) {
                 ok = false;
                 break;
             }
-            if (qq == 0) {
-                const float l_row = sm.qmax[row][0] + sm.qmax[row][1] + sm.qmax[row][2] + sm.qmax[row][3];
-                sm.inv_l[row] = (valid && l_row > 0.f) ? L.v_scale / l_row : 0.f;
-            }
-            softmax_bar();
+            sm.lsum[ob][row][qq] = l_part;
+            warp_arrive(&sm.l_full[ob], lane);
+            ++nact;
+        }
+    } else {
+        // ---------------- epilogue (128 threads, warps 16-19) ----------------
+        // Warp e reads TMEM lane quadrant e: thread (e, lane) holds head dimension 32 e + lane of
+        // every row, so each row's 32 dimensions leave as one 64-byte store per warp.  Row
+        // metadata (output row index, 1 / l) is computed lane-parallel, 32 rows at a time, and
+        // broadcast with shuffles; no barrier spans the four warps, so each leaves on its own
+        // when a wait gives up.
+        const int eq = warp - kWarpEpi0;
+        const int dim = 32 * eq + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * eq) << 16;
+        uint32_t nact = 0;
+        for (int64_t gi = g0; gi < L.n_groups; gi += gstep) {
+            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
+            if (nU == 0)
+                continue;
+            const int h = L.gmeta[3 * gi + 1];
+            const int R = L.gsize[gi] * L.G;
+            const int npad = (R + 15) & ~15;
+            const uint32_t ob = nact & 1u;
+            if (!warp_wait(&sm.o_full[ob], (nact >> 1) & 1u, &sm.abort_flag, lane) ||
+                !warp_wait(&sm.l_full[ob], (nact >> 1) & 1u, &sm.abort_flag, lane))
+                break;
             tc_fence_after();
-            for (int c0 = 16 * hw; c0 < npad; c0 += 32) {
-                uint32_t ohi[16], olo[16];
-                tmem_ld16(o_addr + c0, ohi);
-                tmem_ld16(o_addr + npad + c0, olo);
-                tmem_ld_wait16(ohi);
-                tmem_ld_wait16(olo);
+            const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
+            for (int cb = 0; cb < npad; cb += 32) {
+                const int r = cb + lane;
+                float inv = 0.f;
+                int32_t orow = 0; // output row index tok * Hq + hq
+                if (r < R) {
+                    const int mi = r / L.G;
+                    const int64_t tok = L.qids[gi * L.g + mi];
+                    orow = static_cast<int32_t>(tok * L.Hq + h * L.G + (r - mi * L.G));
+                    const float l_row = sm.lsum[ob][r][0] + sm.lsum[ob][r][1] + sm.lsum[ob][r][2] + sm.lsum[ob][r][3];
+                    inv = l_row > 0.f ? L.v_scale / l_row : 0.f;
+                }
+                const int cend = min(cb + 32, npad);
+                for (int c0 = cb; c0 < cend; c0 += 16) {
+                    uint32_t ohi[16], olo[16];
+                    tmem_ld16(o_addr + c0, ohi);
+                    tmem_ld16(o_addr + npad + c0, olo);
+                    tmem_ld_wait16(ohi);
+                    tmem_ld_wait16(olo);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int r = c0 + e;
-                    const float val = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * sm.inv_l[r];
-                    sm.out[r * kHeadDim + dlane] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                    for (int e = 0; e < 16; ++e) {
+                        const int src = c0 - cb + e;
+                        const float ie = __shfl_sync(kFull, inv, src);
+                        const int32_t oe = __shfl_sync(kFull, orow, src);
+                        if (c0 + e < R) {
+                            const float val = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * ie;
+                            L.O[static_cast<size_t>(oe) * kHeadDim + dim] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                        }
+                    }
                 }
             }
             tc_fence_before();
             warp_arrive(&sm.o_free[ob], lane);
-            softmax_bar();
-            for (int qn = st; qn < R * 16; qn += kSmThreads) {
-                const int r = qn >> 4, c = qn & 15;
-                uint16_t *dst = L.O + (static_cast<size_t>(sm.row_tok[r]) * L.Hq + sm.row_hq[r]) * kHeadDim;
-                reinterpret_cast<uint4 *>(dst)[c] =
-                    reinterpret_cast<const uint4 *>(sm.out + r * kHeadDim)[c];
-            }
-            softmax_bar(); // row_tok, qmax, inv_l and out are rewritten by the next group
             ++nact;
         }
     }
