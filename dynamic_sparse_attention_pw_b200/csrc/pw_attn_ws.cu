@@ -1,27 +1,38 @@
 // pw_attn_ws.cu -- persistent, warp-specialised ID-aware union attention (tiles of <= 64 rows).
 //
-// Same arithmetic as the one-group-per-CTA kernel in pw_attn.cu ("PageWeaver: KV-Guided Query
+// Same result as the one-group-per-CTA kernel in pw_attn.cu ("PageWeaver: KV-Guided Query
 // Unions for Sparse Attention", Abstract: union pages loaded once per group, each query masked
 // to its own support, complete output per query, FP8 KV), organised so that the tensor-core
 // work of one page overlaps the decode and softmax work of its neighbours.
 //
+// S = Q K^T runs on the FP8 tensor-core path with the E4M3 K page exactly as stored: each Q row
+// is scaled by a power of two and split into two E4M3 parts, q' = q1 + q2, which is exact for
+// every element within 2^9 of the row's largest (an 8-bit bf16 significand is a 4-bit E4M3
+// significand plus a remainder of at most 4 bits); S = (q1 K^T + q2 K^T) 2^-s.  The product
+// O^T = V^T P^T stays on bf16 operands (V decoded exactly, P split into bf16 hi + lo parts).
+//
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
-//   warps 0-7    decode   Q tile of each group (bf16, gathered by query ID); E4M3 K and V
-//                         pages -> bf16 operand tiles
-//   warps 8-15   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
+//   warps 0-3    decode   Q tile of each group (gathered by query ID, scaled, split into two
+//                         E4M3 parts); E4M3 V pages -> bf16 operand tiles
+//   warps 4-11   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
 //                         O^T rescale, per-row sums of each group
-//   warps 16-19  epilogue O^T of a finished group -> bf16 rows of O (one warp per TMEM lane
+//   warps 12-15  epilogue O^T of a finished group -> bf16 rows of O (one warp per TMEM lane
 //                         quadrant), while the softmax warps already work on the next group
-//   warp 20      load     bulk copies (TMA) of the union pages into a 3-stage FP8 ring
-//   warp 21      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
+//   warp 16      load     TMA copies of the union pages: K through a tensor map with the
+//                         128-byte swizzle the MMA reads, V as plain bulk copies
+//   warp 17      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
+// Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
+// its scheduler delays its waits and issues.
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
 // (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, which the
-// epilogue adds.  K and V have separate buffers: a K slot is free once S is done, a V slot
+// epilogue adds.  A K stage is free once S is done, a V stage once it is decoded, a bf16 V slot
 // once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
 // mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
 // other roles.
 #include <cstdint>
+#include <cuda.h> // CUtensorMap and its enums (the encoder itself is fetched at run time)
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "pw_attn_common.cuh"
@@ -33,32 +44,33 @@ namespace {
 
 using namespace attn;
 
-constexpr int kNS = 3;        // FP8 page stages
-constexpr int kNK = 3;        // bf16 K slots
+constexpr int kNSK = 6;       // E4M3 K page stages (operands of S)
+constexpr int kNSV = 6;       // E4M3 V page stages
 constexpr int kNV = 3;        // bf16 V slots
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 128;
 constexpr int kSmThreads = 256;
 constexpr int kEpiThreads = 128;
-constexpr int kWarpSm0 = 8, kWarpEpi0 = 16, kWarpLoad = 20, kWarpMma = 21;
-constexpr int kThreads = 704; // 22 warps
+constexpr int kWarpSm0 = kDecThreads / 32, kWarpEpi0 = kWarpSm0 + 8, kWarpLoad = kWarpEpi0 + 4,
+              kWarpMma = kWarpLoad + 1;
+constexpr int kThreads = 32 * (kWarpMma + 1);
+static_assert(kWarpSm0 % 4 == 0, "softmax warp w must sit in TMEM lane quadrant w % 4");
 static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
 constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 64, O^T[0..1] at 128 / 256
 constexpr uint32_t kColO = 128;
-constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
+constexpr uint32_t kIdescS = idesc_e4m3_f32(64, 64);
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 struct __align__(1024) WsSmem {
-    uint8_t q[2][2][64 * 128];   // [Q buffer][dim-block][64 rows][128 B]
-    uint8_t k[kNK][2][64 * 128]; // [slot][dim-block][64 keys][128 B]
-    uint8_t v[kNV][2][64 * 128];
+    uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
+    uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] bf16, swizzled
     uint8_t p[2][128 * 128];     // [buffer][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
-    uint8_t stage_k[kNS][kPageBytes];
-    uint8_t stage_v[kNS][kPageBytes];
+    uint8_t stage_k[kNSK][kPageBytes]; // E4M3 K pages, 128-byte swizzled by the tensor copy
+    uint8_t stage_v[kNSV][kPageBytes]; // E4M3 V pages, row-major
     float alpha[2][64];
     float qmax[64][4];    // per-row partial maxima exchanged by the row's four threads
     float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
-    uint64_t full_stage[kNS], empty_stage[kNS];
-    uint64_t k_full[kNK], k_empty[kNK];
+    uint64_t kst_full[kNSK], kst_empty[kNSK];
+    uint64_t vst_full[kNSV], vst_empty[kNSV];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
     uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete
     uint64_t s_empty[2];
@@ -68,7 +80,7 @@ struct __align__(1024) WsSmem {
     uint64_t l_full[2]; // row sums of that group published
     uint64_t o_free[2]; // epilogue done with O buffer b (and lsum[b])
     uint64_t drain_bar;
-    uint32_t load_issued; // pages whose copies the load warp issued (for the abort drain)
+    uint32_t k_issued, v_issued; // pages whose K / V copies the load warp issued (abort drain)
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t early_exit;
@@ -79,13 +91,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait that also gives up as soon as another role has aborted.
+// Bounded wait that also gives up as soon as another role has aborted.  The abort flag and the
+// clock are read once per eight tries, so a spinning thread issues little besides the tries.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k)
+            if (mbar_try_wait(bar, parity))
+                return true;
         if (*reinterpret_cast<volatile int32_t *>(abort_flag) != 0)
             return false;
         if (clock64() - t0 > kWaitCycles) {
@@ -93,26 +110,46 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
             return false;
         }
     }
-    return true;
 }
 
-// Named barrier 1 over the 256 softmax threads, returning whether any of them passed `pred`.
-__device__ __forceinline__ bool softmax_bar_or(bool pred)
+// Named barriers, one per role that has more than one warp (0 is __syncthreads).
+constexpr uint32_t kBarSoftmax = 1, kBarDecode = 2, kBarEpilogue = 3;
+
+// Named barrier `id` over `n` threads, returning whether any of them passed `pred`.  Warps
+// blocked here issue nothing, so one thread of a role waits on an mbarrier and the others wait
+// here for its verdict.
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t n, bool pred)
 {
     uint32_t r;
     asm volatile("{\n\t.reg .pred p, q;\n\t"
                  "setp.ne.u32 q, %1, 0;\n\t"
-                 "bar.red.or.pred p, 1, 256, q;\n\t"
+                 "bar.red.or.pred p, %2, %3, q;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}\n"
                  : "=r"(r)
-                 : "r"(pred ? 1u : 0u)
+                 : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
                  : "memory");
     return r != 0;
+}
+
+__device__ __forceinline__ bool softmax_bar_or(bool pred)
+{
+    return bar_or(kBarSoftmax, kSmThreads, pred);
 }
 
 __device__ __forceinline__ void softmax_bar()
 {
     asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
+// One thread of a role (`leader`) waits on the mbarrier; the role's `n` threads learn the
+// outcome at named barrier `id`.  true = the phase completed; false = every thread gives up.
+__device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, int32_t *abort_flag,
+                                          bool leader, uint32_t id, uint32_t n)
+{
+    bool ok = true;
+    if (leader)
+        ok = wait_bar(bar, parity, abort_flag);
+    return !bar_or(id, n, !ok);
 }
 
 // A descriptor's start-address field is (address >> 4) in its low 14 bits: a descriptor for
@@ -130,15 +167,67 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane)
         mbar_arrive(bar);
 }
 
-// Lane 0 waits; the warp follows (lane 0's acquire is passed on by the warp barrier).
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *abort_flag, int lane)
+// ---------------- Q: power-of-two row scale and the exact two-part E4M3 split ----------------
+
+// Largest bf16 exponent field among the eight values packed in v.
+__device__ __forceinline__ uint32_t max_exp8(const uint4 v)
 {
-    int ok = 1;
-    if (lane == 0)
-        ok = wait_bar(bar, parity, abort_flag);
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-    __syncwarp();
-    return ok != 0;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        m = max(m, max((w[i] >> 7) & 0xFFu, (w[i] >> 23) & 0xFFu));
+    return m;
+}
+
+// Scale exponent s of a Q row whose largest bf16 exponent field is e: 2^s brings the row's
+// largest magnitude into [128, 256), inside the E4M3 range (largest finite 448).  Clamped so
+// that 2^s and 2^-s are normal floats.
+__device__ __forceinline__ int q_scale_exp(uint32_t e)
+{
+    return min(max(134 - static_cast<int>(e), -126), 126);
+}
+
+__device__ __forceinline__ float exp2i(int s) // 2^s for s in [-126, 127]
+{
+    return __int_as_float((s + 127) << 23);
+}
+
+// Two f32 -> packed E4M3 pair (round to nearest even); `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi)
+{
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// Packed E4M3 pair -> its two values as f32 (exact).
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t pair, float &lo, float &hi)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(pair)));
+    const __half2 h = *reinterpret_cast<const __half2 *>(&h2);
+    lo = __low2float(h);
+    hi = __high2float(h);
+}
+
+// Eight bf16 values (element 0 in the low half of v.x) times 2^s -> E4M3 parts q1 and q2 with
+// q1 + q2 = q 2^s; byte i of each result holds element i.
+__device__ __forceinline__ void split_q8(const uint4 v, float scale, uint2 &q1, uint2 &q2)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t a[4], b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float x0 = __uint_as_float(w[i] << 16) * scale;
+        const float x1 = __uint_as_float(w[i] & 0xFFFF0000u) * scale;
+        a[i] = e4m3x2_rn(x0, x1);
+        float y0, y1;
+        e4m3x2_to_f32(a[i], y0, y1);
+        b[i] = e4m3x2_rn(x0 - y0, x1 - y1);
+    }
+    q1 = make_uint2(a[0] | (a[1] << 16), a[2] | (a[3] << 16));
+    q2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
 struct PendingPV {
@@ -146,7 +235,10 @@ struct PendingPV {
     bool first, last;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch L)
+// tmap_k: the K pages as a 2-D byte tensor [n_phys * Hkv * 64 rows][128], boxes of 64 x 128
+// with the 128-byte swizzle, so that one copy lands a page as the K-major operand of S.
+__global__ void __launch_bounds__(kThreads, 1)
+    k_union_attn_ws(const AttnLaunch L, const __grid_constant__ CUtensorMap tmap_k)
 {
     extern __shared__ uint8_t smem_raw[];
     WsSmem &sm = *reinterpret_cast<WsSmem *>(
@@ -161,13 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
 
     if (tid == 0) {
         // Arrivals from the decode and softmax roles are one per warp (after __syncwarp).
-        for (int s = 0; s < kNS; ++s) {
-            mbar_init(&sm.full_stage[s], 1);
-            mbar_init(&sm.empty_stage[s], kDecThreads / 32);
+        for (int s = 0; s < kNSK; ++s) {
+            mbar_init(&sm.kst_full[s], 1);
+            mbar_init(&sm.kst_empty[s], 1);
         }
-        for (int s = 0; s < kNK; ++s) {
-            mbar_init(&sm.k_full[s], kDecThreads / 32);
-            mbar_init(&sm.k_empty[s], 1);
+        for (int s = 0; s < kNSV; ++s) {
+            mbar_init(&sm.vst_full[s], 1);
+            mbar_init(&sm.vst_empty[s], kDecThreads / 32);
         }
         for (int s = 0; s < kNV; ++s) {
             mbar_init(&sm.v_full[s], kDecThreads / 32);
@@ -185,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         }
         mbar_init(&sm.drain_bar, 1);
         sm.abort_flag = 0;
-        sm.load_issued = 0;
+        sm.k_issued = 0;
+        sm.v_issued = 0;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -199,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
     const int64_t g0 = blockIdx.x, gstep = gridDim.x;
 
     if (warp == kWarpLoad) {
-        // ---------------- load: union pages -> FP8 stages ----------------
+        // ---------------- load: union pages -> K and V stages ----------------
         uint32_t it = 0;
         bool stop = false;
         for (int64_t gi = g0; gi < L.n_groups && !stop; gi += gstep) {
@@ -220,14 +313,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     const int ph = __shfl_sync(kFull, phys, jj);
                     int ok = 1;
                     if (lane == 0) {
-                        const uint32_t st = it % kNS;
-                        ok = wait_bar(&sm.empty_stage[st], ((it / kNS) & 1u) ^ 1u, &sm.abort_flag);
+                        const uint32_t ks = it % kNSK, vs = it % kNSV;
+                        const int32_t row = (ph * L.Hkv + h) * 64;
+                        ok = wait_bar(&sm.kst_empty[ks], ((it / kNSK) & 1u) ^ 1u, &sm.abort_flag);
                         if (ok) {
-                            const size_t off = (static_cast<size_t>(ph) * L.Hkv + h) * kPageBytes;
-                            mbar_arrive_expect_tx(&sm.full_stage[st], 2 * kPageBytes);
-                            bulk_g2s(sm.stage_k[st], L.K + off, kPageBytes, &sm.full_stage[st]);
-                            bulk_g2s(sm.stage_v[st], L.V + off, kPageBytes, &sm.full_stage[st]);
-                            sm.load_issued = it + 1;
+                            mbar_arrive_expect_tx(&sm.kst_full[ks], kPageBytes);
+                            tma_load_2d(sm.stage_k[ks], &tmap_k, 0, row, &sm.kst_full[ks]);
+                            sm.k_issued = it + 1;
+                            ok = wait_bar(&sm.vst_empty[vs], ((it / kNSV) & 1u) ^ 1u, &sm.abort_flag);
+                        }
+                        if (ok) {
+                            mbar_arrive_expect_tx(&sm.vst_full[vs], kPageBytes);
+                            bulk_g2s(sm.stage_v[vs], L.V + static_cast<size_t>(row) * 128, kPageBytes,
+                                     &sm.vst_full[vs]);
+                            sm.v_issued = it + 1;
                         }
                     }
                     if (__shfl_sync(kFull, ok, 0) == 0) {
@@ -286,28 +385,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 ok = false;
                 break;
             }
-            const uint64_t aq0 = desc_add(dsw, smem_u32(sm.q[qb][0]));
-            const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][1]));
+            const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][0]));
+            const uint64_t aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
             for (int j = 0; j < nU; ++j, ++it) {
-                const uint32_t ks = it % kNK, sb = it & 1u;
-                if (!wwait(&sm.k_full[ks], (it / kNK) & 1u) ||
+                const uint32_t ks = it % kNSK, sb = it & 1u;
+                if (!wwait(&sm.kst_full[ks], (it / kNSK) & 1u) ||
                     !wwait(&sm.s_empty[sb], ((it >> 1) & 1u) ^ 1u)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bk0 = desc_add(dsw, smem_u32(sm.k[ks][0]));
-                const uint64_t bk1 = desc_add(dsw, smem_u32(sm.k[ks][1]));
+                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[ks]));
                 const uint32_t ds = tmem + 64 * sb;
                 if (elect_one()) {
+                    // S' = q1 K^T + q2 K^T: four k-steps of 32 dims for each part
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ss(ds, aq0 + 2u * kk, bk0 + 2u * kk, kIdescS, kk > 0 ? 1u : 0u);
+                        mma_f8_ss(ds, aq1 + 2u * kk, bk + 2u * kk, kIdescS, kk > 0 ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ss(ds, aq1 + 2u * kk, bk1 + 2u * kk, kIdescS, 1u);
+                        mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, kIdescS, 1u);
                     mma_commit(&sm.s_done[sb]);
-                    mma_commit(&sm.k_empty[ks]);
+                    mma_commit(&sm.kst_empty[ks]);
                     if (j == nU - 1)
                         mma_commit(&sm.q_empty[qb]);
                 }
@@ -324,7 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         if (ok && have_prev)
             (void)issue_pv(prev);
     } else if (warp < kWarpSm0) {
-        // ---------------- decode: Q tiles and E4M3 -> bf16 K/V tiles (256 threads) ----------------
+        // ---------------- decode: Q tiles (two E4M3 parts) and E4M3 -> bf16 V tiles ----------------
+        // One thread (tid 0) waits on each mbarrier; the others learn the outcome at named
+        // barrier kBarDecode.
         uint32_t it = 0, nact = 0;
         bool ok = true;
         for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
@@ -334,12 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             if (nU == 0)
                 continue;
             const uint32_t qb = nact & 1u;
-            if (!warp_wait(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag, lane)) {
+            if (!role_wait(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag, tid == 0,
+                           kBarDecode, kDecThreads)) {
                 ok = false;
                 break;
             }
+            // Row r of the tile is query head h G + r % G of token qids[r / G].  Sixteen
+            // consecutive lanes hold one row (eight dims each) and agree on its scale.
 #pragma unroll
-            for (int rep = 0; rep < 4; ++rep) {
+            for (int rep = 0; rep < 1024 / kDecThreads; ++rep) {
                 const int qn = tid + kDecThreads * rep;
                 const int row = qn >> 4, c = qn & 15;
                 uint4 val = make_uint4(0u, 0u, 0u, 0u);
@@ -350,21 +454,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                     val = __ldg(reinterpret_cast<const uint4 *>(
                                     L.Q + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim) + c);
                 }
-                *reinterpret_cast<uint4 *>(sm.q[qb][c >> 3] + swz(row, c & 7)) = val;
+                uint32_t e = max_exp8(val);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1)
+                    e = max(e, __shfl_xor_sync(kFull, e, o));
+                uint2 q1, q2;
+                split_q8(val, exp2i(q_scale_exp(e)), q1, q2);
+                const uint32_t off = swz(row, c >> 1) + 8u * (c & 1);
+                *reinterpret_cast<uint2 *>(sm.q[qb][0] + off) = q1;
+                *reinterpret_cast<uint2 *>(sm.q[qb][1] + off) = q2;
             }
             fence_proxy_async_smem();
             warp_arrive(&sm.q_full[qb], lane);
             for (int j = 0; j < nU; ++j, ++it) {
-                const uint32_t st = it % kNS, ks = it % kNK, vs = it % kNV;
-                if (!warp_wait(&sm.full_stage[st], (it / kNS) & 1u, &sm.abort_flag, lane) ||
-                    !warp_wait(&sm.k_empty[ks], ((it / kNK) & 1u) ^ 1u, &sm.abort_flag, lane)) {
-                    ok = false;
-                    break;
-                }
-                decode_page<kDecThreads>(sm.stage_k[st], sm.k[ks], tid);
-                fence_proxy_async_smem();
-                warp_arrive(&sm.k_full[ks], lane);
-                if (!warp_wait(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag, lane)) {
+                const uint32_t st = it % kNSV, vs = it % kNV;
+                bool got = true;
+                if (tid == 0)
+                    got = wait_bar(&sm.vst_full[st], (it / kNSV) & 1u, &sm.abort_flag) &&
+                          wait_bar(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag);
+                if (bar_or(kBarDecode, kDecThreads, !got)) {
                     ok = false;
                     break;
                 }
@@ -373,19 +481,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&sm.v_full[vs]);
-                    mbar_arrive(&sm.empty_stage[st]);
+                    mbar_arrive(&sm.vst_empty[st]);
                 }
             }
             ++nact;
         }
     } else if (warp < kWarpEpi0) {
-        // ---------------- softmax (256 threads, warps 8-15) ----------------
+        // ---------------- softmax (256 threads) ----------------
         // Four threads share a row: warp (quadrant qd, half hw) reads TMEM lanes of rows
         // 16 qd .. 16 qd + 15 and keys 32 hw .. 32 hw + 31; lane / 16 picks 16 of those keys.
         // A row's running max m is identical in its four threads and changes only on the slow
         // path, which runs when some element of some row exceeds its m by more than 2^8 (one
         // OR over all 256 threads decides), so the common path needs no exchange.
         const int sw = warp - kWarpSm0;     // 0..7
+        const bool sleader = sw == 0 && lane == 0; // the role's one mbarrier waiter
         const int qd = sw & 3;              // TMEM lane quadrant
         const int hw = sw >> 2;             // key half of the page read by this warp
         const int row = 16 * qd + (lane & 15);
@@ -404,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         uint32_t pv_done = 0;
         auto wait_pv = [&](uint32_t x) -> bool { // product of page x complete
             for (; pv_done <= x; ++pv_done)
-                if (lane == 0 && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
+                if (sleader && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
                     return false;
             return true;
         };
@@ -425,6 +534,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 pos = static_cast<int>(tok - L.cu[b]);
                 own = pos >> 6;
                 bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
+            }
+            // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain
+            // factor.  s is recomputed here from the row exactly as the decode warps did.
+            float crow_r = crow, acrow_r = acrow;
+            if (valid && nU > 0) {
+                const uint4 *qrow = reinterpret_cast<const uint4 *>(
+                    L.Q + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim);
+                uint32_t e = 0;
+#pragma unroll 4
+                for (int c = 0; c < 16; ++c)
+                    e = max(e, max_exp8(__ldg(qrow + c)));
+                const float inv = exp2i(-q_scale_exp(e));
+                crow_r = crow * inv;
+                acrow_r = acrow * inv;
             }
             if (nU == 0) {
                 if (valid) { // no union page: every row of the group is empty
@@ -451,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 const uint32_t sb = it & 1u, pb = it & 1u;
                 // every abort decision of this role is collective: a thread that left alone
                 // would strand the others at the named barrier or in a warp-wide TMEM load
-                ok = lane != 0 || wait_bar(&sm.s_done[sb], (it >> 1) & 1u, &sm.abort_flag);
+                ok = !sleader || wait_bar(&sm.s_done[sb], (it >> 1) & 1u, &sm.abort_flag);
                 if (softmax_bar_or(!ok)) {
                     ok = false;
                     break;
@@ -482,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                             lm = fmaxf(lm, -__uint_as_float(sv[e]));
                 }
                 if (nq > 0)
-                    lm *= acrow;
+                    lm *= acrow_r;
                 if (softmax_bar_or(nq > 0 && lm > m_used + kRescaleLog2)) {
                     // slow path: the row's four threads agree on its max
                     sm.qmax[row][qq] = lm;
@@ -532,16 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 if (__all_sync(kFull, nq == 16)) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), crow, negm));
-                        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow, negm));
+                        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), crow_r, negm));
+                        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow_r, negm));
                         l_part += p0 + p1;
                         split_pair(p0, p1, hi[e], lo[e]);
                     }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), crow, negm)) : 0.f;
-                        const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow, negm)) : 0.f;
+                        const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), crow_r, negm)) : 0.f;
+                        const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow_r, negm)) : 0.f;
                         l_part += p0 + p1;
                         split_pair(p0, p1, hi[e], lo[e]);
                     }
@@ -564,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
                 break;
             // Publish the row-sum partials of this group for the epilogue warps.  lsum[ob] was
             // last read by the epilogue of group nact - 2, which released it with o_free[ob].
-            ok = lane != 0 || wait_bar(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
+            ok = !sleader || wait_bar(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
             if (softmax_bar_or(!ok)) {
                 ok = false;
                 break;
@@ -574,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             ++nact;
         }
     } else {
-        // ---------------- epilogue (128 threads, warps 16-19) ----------------
+        // ---------------- epilogue (128 threads) ----------------
         // Warp e reads TMEM lane quadrant e: thread (e, lane) holds head dimension 32 e + lane of
         // every row, so each row's 32 dimensions leave as one 64-byte store per warp.  Row
         // metadata (output row index, 1 / l) is computed lane-parallel, 32 rows at a time, and
@@ -592,8 +715,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
             const int R = L.gsize[gi] * L.G;
             const int npad = (R + 15) & ~15;
             const uint32_t ob = nact & 1u;
-            if (!warp_wait(&sm.o_full[ob], (nact >> 1) & 1u, &sm.abort_flag, lane) ||
-                !warp_wait(&sm.l_full[ob], (nact >> 1) & 1u, &sm.abort_flag, lane))
+            bool got = true;
+            if (eq == 0 && lane == 0)
+                got = wait_bar(&sm.o_full[ob], (nact >> 1) & 1u, &sm.abort_flag) &&
+                      wait_bar(&sm.l_full[ob], (nact >> 1) & 1u, &sm.abort_flag);
+            if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 break;
             tc_fence_after();
             const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
@@ -641,10 +767,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
         // Let copies and products still in flight land before the CTA exits (bounded waits):
         // the last copy issued on each stage, and every product issued so far.
         if (tid == 0) {
-            const uint32_t n = sm.load_issued;
-            for (uint32_t s = 0; s < kNS && s < n; ++s) {
-                const uint32_t last = s + ((n - 1 - s) / kNS) * kNS;
-                (void)mbar_wait(&sm.full_stage[s], (last / kNS) & 1u);
+            const uint32_t nk = sm.k_issued, nv = sm.v_issued;
+            for (uint32_t s = 0; s < kNSK && s < nk; ++s) {
+                const uint32_t last = s + ((nk - 1 - s) / kNSK) * kNSK;
+                (void)mbar_wait(&sm.kst_full[s], (last / kNSK) & 1u);
+            }
+            for (uint32_t s = 0; s < kNSV && s < nv; ++s) {
+                const uint32_t last = s + ((nv - 1 - s) / kNSV) * kNSV;
+                (void)mbar_wait(&sm.vst_full[s], (last / kNSV) & 1u);
             }
         }
         if (warp == kWarpMma) {
@@ -664,10 +794,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_union_attn_ws(const AttnLaunch 
 
 } // namespace
 
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no link to libcuda).
+EncodeTiledFn encode_tiled()
+{
+    static const EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+} // namespace
+
 cudaError_t attn_ws_launch(const AttnLaunch &L, cudaStream_t st)
 {
     if (L.n_groups == 0)
         return cudaSuccess;
+    // Page rows are addressed with 32-bit tensor coordinates.
+    const uint64_t k_rows = static_cast<uint64_t>(L.n_phys) * L.Hkv * 64;
+    if (L.n_phys < 1 || k_rows > 0x7FFFFFFFull)
+        return cudaErrorInvalidValue;
+    const EncodeTiledFn enc = encode_tiled();
+    if (enc == nullptr)
+        return cudaErrorNotSupported;
+    CUtensorMap tmap_k;
+    const cuuint64_t dims[2] = {128, k_rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, 64};
+    const cuuint32_t estrides[2] = {1, 1};
+    if (enc(&tmap_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(L.K), dims, strides,
+            box, estrides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
@@ -680,7 +849,7 @@ cudaError_t attn_ws_launch(const AttnLaunch &L, cudaStream_t st)
     if (e != cudaSuccess)
         return e;
     const int64_t grid = L.n_groups < sms ? L.n_groups : sms;
-    k_union_attn_ws<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(L);
+    k_union_attn_ws<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(L, tmap_k);
     return cudaGetLastError();
 }
 
