@@ -342,10 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // operands are computed by the converged warp (uniform registers), the elected lane
         // (always lane 0) issues the MMAs and their commits.
         auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            int ok = 1;
-            if (lane == 0)
-                ok = wait_bar(bar, parity, &sm.abort_flag);
-            return __shfl_sync(kFull, ok, 0) != 0;
+            const bool ok = wait_bar(bar, parity, &sm.abort_flag); // every lane polls
+            return __all_sync(kFull, ok);
         };
         const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
         const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // MN-major V^T
