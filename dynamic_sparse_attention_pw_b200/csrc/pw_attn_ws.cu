@@ -44,8 +44,9 @@ namespace {
 
 using namespace attn;
 
-constexpr int kNSK = 6;       // E4M3 K page stages (operands of S)
-constexpr int kNSV = 6;       // E4M3 V page stages
+constexpr int kNSK = 5;       // E4M3 K page stages (operands of S)
+constexpr int kNSV = 5;       // E4M3 V page stages
+constexpr int kNJ = 3;        // group records in flight
 constexpr int kNV = 3;        // bf16 V slots
 constexpr int kDecThreads = 128;
 constexpr int kSmThreads = 256;
@@ -60,15 +61,29 @@ constexpr uint32_t kColO = 128;
 constexpr uint32_t kIdescS = idesc_e4m3_f32(64, 64);
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
+// One group as the load warp hands it to the other roles, so that none of them meets a chain
+// of dependent global loads when it starts a group.
+struct GroupJob {
+    int32_t tok[64];    // query token of each tile row (rows >= R: 0)
+    int32_t pos[64];    // its position within its sequence
+    int32_t qexp[64];   // its Q scale exponent (written by the decode warps)
+    uint32_t word0[32]; // per query of the group: its membership word of the first union page
+    int32_t b, h, R, nU, u0, pg0; // nU < 0: no further group
+};
+
 struct __align__(1024) WsSmem {
     uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
     uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] bf16, swizzled
     uint8_t p[2][128 * 128];     // [buffer][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
     uint8_t stage_k[kNSK][kPageBytes]; // E4M3 K pages, 128-byte swizzled by the tensor copy
     uint8_t stage_v[kNSV][kPageBytes]; // E4M3 V pages, row-major
+    uint8_t q_raw[64 * 256];           // bf16 Q rows of the next group, row r at 256 r
+    GroupJob job[kNJ];
     float alpha[2][64];
     float qmax[64][4];    // per-row partial maxima exchanged by the row's four threads
     float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
+    uint64_t job_full[kNJ], job_empty[kNJ];
+    uint64_t qraw_full, qraw_empty;
     uint64_t kst_full[kNSK], kst_empty[kNSK];
     uint64_t vst_full[kNSV], vst_empty[kNSV];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
@@ -81,6 +96,7 @@ struct __align__(1024) WsSmem {
     uint64_t o_free[2]; // epilogue done with O buffer b (and lsum[b])
     uint64_t drain_bar;
     uint32_t k_issued, v_issued; // pages whose K / V copies the load warp issued (abort drain)
+    uint32_t q_issued;           // groups whose Q rows it copied
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t early_exit;
@@ -253,6 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         // Arrivals from the decode and softmax roles are one per warp (after __syncwarp).
+        for (int s = 0; s < kNJ; ++s) {
+            mbar_init(&sm.job_full[s], 1);
+            mbar_init(&sm.job_empty[s], kDecThreads / 32 + 1 + kSmThreads / 32);
+        }
+        mbar_init(&sm.qraw_full, 1);
+        mbar_init(&sm.qraw_empty, kDecThreads / 32);
         for (int s = 0; s < kNSK; ++s) {
             mbar_init(&sm.kst_full[s], 1);
             mbar_init(&sm.kst_empty[s], 1);
@@ -279,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.abort_flag = 0;
         sm.k_issued = 0;
         sm.v_issued = 0;
+        sm.q_issued = 0;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -292,12 +315,78 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t g0 = blockIdx.x, gstep = gridDim.x;
 
     if (warp == kWarpLoad) {
-        // ---------------- load: union pages -> K and V stages ----------------
-        uint32_t it = 0;
+        // ---------------- load: group records, Q rows, union pages -> stages ----------------
+        // Runs pages ahead of the other roles, so the latency of its dependent global loads
+        // (group -> query IDs -> positions and membership words) stays off their path.  Every
+        // lane polls its mbarriers; lane 0 issues the page copies.
+        auto lwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(kFull, wait_bar(bar, parity, &sm.abort_flag));
+        };
+        uint32_t it = 0, nj = 0;
         bool stop = false;
         for (int64_t gi = g0; gi < L.n_groups && !stop; gi += gstep) {
             const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
+            const int gsz = L.gsize[gi], R = gsz * L.G;
             const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
+            if (nU == 0) {
+                // no union page: every row of the group is empty
+                for (int idx = lane; idx < R * 16; idx += 32) {
+                    const int r = idx >> 4, c = idx & 15, mi = r / L.G;
+                    const int64_t tok = L.qids[gi * L.g + mi];
+                    const int hq = h * L.G + (r - mi * L.G);
+                    reinterpret_cast<uint4 *>(L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim)[c] =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
+            // the group record
+            const int32_t tok_l = lane < gsz ? L.qids[gi * L.g + lane] : 0;
+            const int32_t cu_b = L.cu[b];
+            const int pg0 = L.union_pages[u0];
+            const uint32_t word0_l =
+                lane < gsz ? __ldg(L.bits + (static_cast<size_t>(tok_l) * L.Hkv + h) * L.words + (pg0 >> 5)) : 0u;
+            const uint32_t jb = nj % kNJ;
+            if (!lwait(&sm.job_empty[jb], ((nj / kNJ) & 1u) ^ 1u)) {
+                stop = true;
+                break;
+            }
+            GroupJob &J = sm.job[jb];
+#pragma unroll
+            for (int r0 = 0; r0 < 64; r0 += 32) {
+                const int r = r0 + lane;
+                const int mi = min(r / L.G, 31);
+                const int32_t t = __shfl_sync(kFull, tok_l, mi);
+                J.tok[r] = r < R ? t : 0;
+                J.pos[r] = r < R ? t - cu_b : 0;
+            }
+            J.word0[lane] = word0_l;
+            if (lane == 0) {
+                J.b = b;
+                J.h = h;
+                J.R = R;
+                J.nU = nU;
+                J.u0 = u0;
+                J.pg0 = pg0;
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.job_full[jb]);
+            // the group's Q rows: query qi's G heads are G consecutive rows of Q
+            if (!lwait(&sm.qraw_empty, (nj & 1u) ^ 1u)) {
+                stop = true;
+                break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.qraw_full, static_cast<uint32_t>(R) * 256u);
+                sm.q_issued = nj + 1;
+            }
+            __syncwarp();
+            if (lane < gsz)
+                bulk_g2s(sm.q_raw + lane * L.G * 256,
+                         L.Q + (static_cast<size_t>(tok_l) * L.Hq + h * L.G) * kHeadDim,
+                         static_cast<uint32_t>(L.G) * 256u, &sm.qraw_full);
+            ++nj;
+            // the union pages
             for (int j0 = 0; j0 < nU && !stop; j0 += 32) {
                 int phys = 0;
                 if (j0 + lane < nU) {
@@ -311,28 +400,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int cnt = min(32, nU - j0);
                 for (int jj = 0; jj < cnt; ++jj, ++it) {
                     const int ph = __shfl_sync(kFull, phys, jj);
-                    int ok = 1;
-                    if (lane == 0) {
-                        const uint32_t ks = it % kNSK, vs = it % kNSV;
-                        const int32_t row = (ph * L.Hkv + h) * 64;
-                        ok = wait_bar(&sm.kst_empty[ks], ((it / kNSK) & 1u) ^ 1u, &sm.abort_flag);
-                        if (ok) {
-                            mbar_arrive_expect_tx(&sm.kst_full[ks], kPageBytes);
-                            tma_load_2d(sm.stage_k[ks], &tmap_k, 0, row, &sm.kst_full[ks]);
-                            sm.k_issued = it + 1;
-                            ok = wait_bar(&sm.vst_empty[vs], ((it / kNSV) & 1u) ^ 1u, &sm.abort_flag);
-                        }
-                        if (ok) {
-                            mbar_arrive_expect_tx(&sm.vst_full[vs], kPageBytes);
-                            bulk_g2s(sm.stage_v[vs], L.V + static_cast<size_t>(row) * 128, kPageBytes,
-                                     &sm.vst_full[vs]);
-                            sm.v_issued = it + 1;
-                        }
-                    }
-                    if (__shfl_sync(kFull, ok, 0) == 0) {
+                    const uint32_t ks = it % kNSK, vs = it % kNSV;
+                    const int32_t row = (ph * L.Hkv + h) * 64;
+                    if (!lwait(&sm.kst_empty[ks], ((it / kNSK) & 1u) ^ 1u)) {
                         stop = true;
                         break;
                     }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sm.kst_full[ks], kPageBytes);
+                        tma_load_2d(sm.stage_k[ks], &tmap_k, 0, row, &sm.kst_full[ks]);
+                        sm.k_issued = it + 1;
+                    }
+                    if (!lwait(&sm.vst_empty[vs], ((it / kNSV) & 1u) ^ 1u)) {
+                        stop = true;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sm.vst_full[vs], kPageBytes);
+                        bulk_g2s(sm.stage_v[vs], L.V + static_cast<size_t>(row) * 128, kPageBytes,
+                                 &sm.vst_full[vs]);
+                        sm.v_issued = it + 1;
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        if (!stop) { // end marker
+            const uint32_t jb = nj % kNJ;
+            if (lwait(&sm.job_empty[jb], ((nj / kNJ) & 1u) ^ 1u)) {
+                if (lane == 0) {
+                    sm.job[jb].nU = -1;
+                    mbar_arrive(&sm.job_full[jb]);
                 }
             }
         }
@@ -372,12 +470,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             return true;
         };
-        for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
-            const int R = L.gsize[gi] * L.G;
+        for (;;) {
+            const uint32_t jb = nact % kNJ;
+            if (!wwait(&sm.job_full[jb], (nact / kNJ) & 1u)) {
+                ok = false;
+                break;
+            }
+            const int R = sm.job[jb].R, nU = sm.job[jb].nU;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.job_empty[jb]);
+            if (nU < 0)
+                break;
             const uint32_t npad = static_cast<uint32_t>((R + 15) & ~15);
-            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
-            if (nU == 0)
-                continue;
             const uint32_t qb = nact & 1u;
             if (!wwait(&sm.q_full[qb], (nact >> 1) & 1u)) {
                 ok = false;
@@ -416,6 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0, j == nU - 1};
                 have_prev = true;
             }
+            if (!ok)
+                break;
             ++nact;
         }
         if (ok && have_prev)
@@ -426,44 +533,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         // barrier kBarDecode.
         uint32_t it = 0, nact = 0;
         bool ok = true;
-        for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
-            const int h = L.gmeta[3 * gi + 1];
-            const int R = L.gsize[gi] * L.G;
-            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
-            if (nU == 0)
-                continue;
-            const uint32_t qb = nact & 1u;
-            if (!role_wait(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag, tid == 0,
-                           kBarDecode, kDecThreads)) {
+        for (;;) {
+            const uint32_t jb = nact % kNJ, qb = nact & 1u;
+            if (!role_wait(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag, tid == 0, kBarDecode,
+                           kDecThreads)) {
                 ok = false;
                 break;
             }
-            // Row r of the tile is query head h G + r % G of token qids[r / G].  Sixteen
-            // consecutive lanes hold one row (eight dims each) and agree on its scale.
+            GroupJob &J = sm.job[jb];
+            const int R = J.R, nU = J.nU;
+            if (nU < 0) {
+                warp_arrive(&sm.job_empty[jb], lane);
+                break;
+            }
+            // Q tile buffer qb was last read by the last S of group nact - 2; the raw rows of
+            // this group have landed.
+            bool got = true;
+            if (tid == 0)
+                got = wait_bar(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag) &&
+                      wait_bar(&sm.qraw_full, nact & 1u, &sm.abort_flag);
+            if (bar_or(kBarDecode, kDecThreads, !got)) {
+                ok = false;
+                break;
+            }
+            // Row r of the tile is query head h G + r % G of query r / G.  Sixteen consecutive
+            // lanes hold one row (eight dims each) and agree on its scale.
 #pragma unroll
             for (int rep = 0; rep < 1024 / kDecThreads; ++rep) {
                 const int qn = tid + kDecThreads * rep;
                 const int row = qn >> 4, c = qn & 15;
-                uint4 val = make_uint4(0u, 0u, 0u, 0u);
-                if (row < R) {
-                    const int mi = row / L.G;
-                    const int64_t tok = L.qids[gi * L.g + mi];
-                    const int hq = h * L.G + (row - mi * L.G);
-                    val = __ldg(reinterpret_cast<const uint4 *>(
-                                    L.Q + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim) + c);
-                }
+                const uint4 val = row < R ? *reinterpret_cast<const uint4 *>(sm.q_raw + row * 256 + c * 16)
+                                          : make_uint4(0u, 0u, 0u, 0u);
                 uint32_t e = max_exp8(val);
 #pragma unroll
                 for (int o = 8; o > 0; o >>= 1)
                     e = max(e, __shfl_xor_sync(kFull, e, o));
+                const int sexp = q_scale_exp(e);
                 uint2 q1, q2;
-                split_q8(val, exp2i(q_scale_exp(e)), q1, q2);
+                split_q8(val, exp2i(sexp), q1, q2);
                 const uint32_t off = swz(row, c >> 1) + 8u * (c & 1);
                 *reinterpret_cast<uint2 *>(sm.q[qb][0] + off) = q1;
                 *reinterpret_cast<uint2 *>(sm.q[qb][1] + off) = q2;
+                if (c == 0)
+                    J.qexp[row] = sexp;
             }
             fence_proxy_async_smem();
             warp_arrive(&sm.q_full[qb], lane);
+            warp_arrive(&sm.qraw_empty, lane);
+            warp_arrive(&sm.job_empty[jb], lane);
             for (int j = 0; j < nU; ++j, ++it) {
                 const uint32_t st = it % kNSV, vs = it % kNV;
                 bool got = true;
@@ -482,6 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&sm.vst_empty[st]);
                 }
             }
+            if (!ok)
+                break;
             ++nact;
         }
     } else if (warp < kWarpEpi0) {
@@ -516,52 +635,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
         bool ok = true;
-        for (int64_t gi = g0; gi < L.n_groups && ok; gi += gstep) {
-            const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
-            const int R = L.gsize[gi] * L.G;
+        for (;;) {
+            // the group record; its Q scale exponents are written with the Q tile
+            const uint32_t jb = nact % kNJ;
+            bool got = true;
+            if (sleader) {
+                got = wait_bar(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag);
+                if (got && sm.job[jb].nU >= 0)
+                    got = wait_bar(&sm.q_full[nact & 1u], (nact >> 1) & 1u, &sm.abort_flag);
+            }
+            if (softmax_bar_or(!got)) {
+                ok = false;
+                break;
+            }
+            const GroupJob &J = sm.job[jb];
+            const int nU = J.nU;
+            if (nU < 0)
+                break;
+            const int h = J.h, R = J.R, u0 = J.u0;
             const int npad = (R + 15) & ~15;
-            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
             const bool valid = row < R;
-            int64_t tok = 0;
-            int hq = 0, pos = 0, own = 0;
-            const uint32_t *bitrow = nullptr;
-            if (valid) {
-                const int mi = row / L.G;
-                tok = L.qids[gi * L.g + mi];
-                hq = h * L.G + (row - mi * L.G);
-                pos = static_cast<int>(tok - L.cu[b]);
-                own = pos >> 6;
-                bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
-            }
-            // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain
-            // factor.  s is recomputed here from the row exactly as the decode warps did.
-            float crow_r = crow, acrow_r = acrow;
-            if (valid && nU > 0) {
-                const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                    L.Q + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim);
-                uint32_t e = 0;
-#pragma unroll 4
-                for (int c = 0; c < 16; ++c)
-                    e = max(e, max_exp8(__ldg(qrow + c)));
-                const float inv = exp2i(-q_scale_exp(e));
-                crow_r = crow * inv;
-                acrow_r = acrow * inv;
-            }
-            if (nU == 0) {
-                if (valid) { // no union page: every row of the group is empty
-                    uint4 *dst = reinterpret_cast<uint4 *>(
-                        L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim + 32 * qq);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        dst[c] = make_uint4(0u, 0u, 0u, 0u);
-                }
-                continue;
-            }
+            const int32_t tok = J.tok[row];
+            const int pos = J.pos[row], own = pos >> 6;
+            const uint32_t *bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
+            // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain factor
+            const float inv = exp2i(-J.qexp[row]);
+            const float crow_r = crow * inv, acrow_r = acrow * inv;
+            int pg_next = J.pg0;
+            uint32_t word_next = valid ? J.word0[row / L.G] : 0u;
+            warp_arrive(&sm.job_empty[jb], lane);
             const uint32_t ob = nact & 1u;
             const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
             float m_used = -INFINITY, l_part = 0.f;
-            int pg_next = L.union_pages[u0];
-            uint32_t word_next = valid ? __ldg(bitrow + (pg_next >> 5)) : 0u;
             for (int j = 0; j < nU; ++j, ++it) {
                 const int pg = pg_next;
                 const uint32_t word = word_next;
@@ -774,6 +879,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t last = s + ((nv - 1 - s) / kNSV) * kNSV;
                 (void)mbar_wait(&sm.vst_full[s], (last / kNSV) & 1u);
             }
+            if (sm.q_issued > 0)
+                (void)mbar_wait(&sm.qraw_full, (sm.q_issued - 1) & 1u);
         }
         if (warp == kWarpMma) {
             if (elect_one()) {
