@@ -88,7 +88,6 @@ struct __align__(1024) WsSmem {
     uint64_t vst_full[kNSV], vst_empty[kNSV];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
     uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete
-    uint64_t s_empty[2];
     uint64_t p_full[2];
     uint64_t q_full[2], q_empty[2];
     uint64_t o_full[2]; // last product of the group in O buffer b complete
@@ -289,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_done[s], 1);
-            mbar_init(&sm.s_empty[s], kSmThreads / 32);
             mbar_init(&sm.p_full[s], kSmThreads / 32);
             mbar_init(&sm.q_full[s], kDecThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
@@ -492,8 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
             for (int j = 0; j < nU; ++j, ++it) {
                 const uint32_t ks = it % kNSK, sb = it & 1u;
-                if (!wwait(&sm.kst_full[ks], (it / kNSK) & 1u) ||
-                    !wwait(&sm.s_empty[sb], ((it >> 1) & 1u) ^ 1u)) {
+                // S buffer sb was last read by the softmax of page it - 2, before it wrote the P
+                // that the product issued in the previous iteration waited for.
+                if (!wwait(&sm.kst_full[ks], (it / kNSK) & 1u)) {
                     ok = false;
                     break;
                 }
@@ -689,7 +688,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_16x32bx2_x16(tmem + lane_base + 64 * sb + 32 * hw, sv);
                 tmem_ld_wait16(sv);
                 tc_fence_before();
-                warp_arrive(&sm.s_empty[sb], lane);
 
                 int n_allow = 0;
                 if ((word >> (pg & 31)) & 1u)
