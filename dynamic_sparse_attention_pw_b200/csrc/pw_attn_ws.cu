@@ -44,8 +44,8 @@ namespace {
 
 using namespace attn;
 
-constexpr int kNSK = 5;       // E4M3 K page stages (operands of S)
-constexpr int kNSV = 5;       // E4M3 V page stages
+constexpr int kNKP = 2;       // E4M3 K stage pairs (one S step each)
+constexpr int kNSV = 3;       // E4M3 V page stages
 constexpr int kNJ = 3;        // group records in flight
 constexpr int kNV = 3;        // bf16 V slots
 constexpr int kDecThreads = 128;
@@ -56,9 +56,9 @@ constexpr int kWarpSm0 = kDecThreads / 32, kWarpEpi0 = kWarpSm0 + 8, kWarpLoad =
 constexpr int kThreads = 32 * (kWarpMma + 1);
 static_assert(kWarpSm0 % 4 == 0, "softmax warp w must sit in TMEM lane quadrant w % 4");
 static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
-constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 64, O^T[0..1] at 128 / 256
-constexpr uint32_t kColO = 128;
-constexpr uint32_t kIdescS = idesc_e4m3_f32(64, 64);
+constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 128, O^T[0..1] at 256 / 384
+constexpr uint32_t kColS = 128;     // one S step: two pages of 64 keys
+constexpr uint32_t kColO = 256;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // One group as the load warp hands it to the other roles, so that none of them meets a chain
@@ -67,15 +67,18 @@ struct GroupJob {
     int32_t tok[64];    // query token of each tile row (rows >= R: 0)
     int32_t pos[64];    // its position within its sequence
     int32_t qexp[64];   // its Q scale exponent (written by the decode warps)
-    uint32_t word0[32]; // per query of the group: its membership word of the first union page
-    int32_t b, h, R, nU, u0, pg0; // nU < 0: no further group
+    uint32_t word0[2][32]; // per query: its membership words of the first two union pages
+    int32_t b, h, R, nU, u0, pg0, pg1; // nU < 0: no further group
 };
 
 struct __align__(1024) WsSmem {
     uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
     uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] bf16, swizzled
-    uint8_t p[2][128 * 128];     // [buffer][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
-    uint8_t stage_k[kNSK][kPageBytes]; // E4M3 K pages, 128-byte swizzled by the tensor copy
+    // [step parity][page of the step][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
+    uint8_t p[2][2][128 * 128];
+    // E4M3 K pages, 128-byte swizzled by the tensor copy; the two pages of a step sit in one
+    // pair, so that they form one 128-row operand
+    uint8_t stage_k[kNKP][2][kPageBytes];
     uint8_t stage_v[kNSV][kPageBytes]; // E4M3 V pages, row-major
     uint8_t q_raw[64 * 256];           // bf16 Q rows of the next group, row r at 256 r
     GroupJob job[kNJ];
@@ -84,17 +87,17 @@ struct __align__(1024) WsSmem {
     float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
     uint64_t job_full[kNJ], job_empty[kNJ];
     uint64_t qraw_full, qraw_empty;
-    uint64_t kst_full[kNSK], kst_empty[kNSK];
+    uint64_t kst_full[kNKP], kst_empty[kNKP];
     uint64_t vst_full[kNSV], vst_empty[kNSV];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
-    uint64_t s_done[2];                 // s_done[i % 2]: S of page i complete
-    uint64_t p_full[2];
+    uint64_t s_done[2];                 // s_done[n % 2]: S of step n complete
+    uint64_t p_full[2];                 // p_full[n % 2]: P of both pages of step n written
     uint64_t q_full[2], q_empty[2];
     uint64_t o_full[2]; // last product of the group in O buffer b complete
     uint64_t l_full[2]; // row sums of that group published
     uint64_t o_free[2]; // epilogue done with O buffer b (and lsum[b])
     uint64_t drain_bar;
-    uint32_t k_issued, v_issued; // pages whose K / V copies the load warp issued (abort drain)
+    uint32_t k_issued, v_issued; // steps / pages whose K / V copies the load warp issued
     uint32_t q_issued;           // groups whose Q rows it copied
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -245,10 +248,61 @@ __device__ __forceinline__ void split_q8(const uint4 v, float scale, uint2 &q1, 
     q2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
-struct PendingPV {
-    uint32_t it, vs, ob, nact, npad;
-    bool first, last;
-};
+// Largest of the first nq of 16 scores, sign-flipped when the log2-domain factor is negative.
+__device__ __forceinline__ float quarter_max(const uint32_t (&sv)[16], int nq, bool flip)
+{
+    float lm = -INFINITY;
+    if (!flip) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (e < nq)
+                lm = fmaxf(lm, __uint_as_float(sv[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (e < nq)
+                lm = fmaxf(lm, -__uint_as_float(sv[e]));
+    }
+    return lm;
+}
+
+// P of 16 keys of one row (the first nq allowed, the rest 0) into rows `row` (P_hi) and
+// npad + row (P_lo) of a page's P buffer; returns their sum.  Only rows < npad write.
+__device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float c, float negm,
+                                        uint8_t *buf, int row, int qq, int npad)
+{
+    uint32_t hi[8], lo[8];
+    float sum = 0.f;
+    if (__all_sync(0xFFFFFFFFu, nq == 16)) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm));
+            sum += p0 + p1;
+            split_pair(p0, p1, hi[e], lo[e]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm)) : 0.f;
+            const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm)) : 0.f;
+            sum += p0 + p1;
+            split_pair(p0, p1, hi[e], lo[e]);
+        }
+    }
+    if (row < npad) {
+        uint8_t *phi = buf, *plo = buf + npad * 128;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t o = swz(row, 2 * qq + cc);
+            *reinterpret_cast<uint4 *>(phi + o) =
+                make_uint4(hi[4 * cc], hi[4 * cc + 1], hi[4 * cc + 2], hi[4 * cc + 3]);
+            *reinterpret_cast<uint4 *>(plo + o) =
+                make_uint4(lo[4 * cc], lo[4 * cc + 1], lo[4 * cc + 2], lo[4 * cc + 3]);
+        }
+    }
+    return sum;
+}
 
 // tmap_k: the K pages as a 2-D byte tensor [n_phys * Hkv * 64 rows][128], boxes of 64 x 128
 // with the 128-byte swizzle, so that one copy lands a page as the K-major operand of S.
@@ -274,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.qraw_full, 1);
         mbar_init(&sm.qraw_empty, kDecThreads / 32);
-        for (int s = 0; s < kNSK; ++s) {
+        for (int s = 0; s < kNKP; ++s) {
             mbar_init(&sm.kst_full[s], 1);
             mbar_init(&sm.kst_empty[s], 1);
         }
@@ -320,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto lwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             return __all_sync(kFull, wait_bar(bar, parity, &sm.abort_flag));
         };
-        uint32_t it = 0, nj = 0;
+        uint32_t it = 0, stp = 0, nj = 0;
         bool stop = false;
         for (int64_t gi = g0; gi < L.n_groups && !stop; gi += gstep) {
             const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
@@ -340,9 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the group record
             const int32_t tok_l = lane < gsz ? L.qids[gi * L.g + lane] : 0;
             const int32_t cu_b = L.cu[b];
-            const int pg0 = L.union_pages[u0];
-            const uint32_t word0_l =
-                lane < gsz ? __ldg(L.bits + (static_cast<size_t>(tok_l) * L.Hkv + h) * L.words + (pg0 >> 5)) : 0u;
+            const int pg0 = L.union_pages[u0], pg1 = nU > 1 ? L.union_pages[u0 + 1] : pg0;
+            const uint32_t *bitrow_l = L.bits + (static_cast<size_t>(tok_l) * L.Hkv + h) * L.words;
+            const uint32_t word0_l = lane < gsz ? __ldg(bitrow_l + (pg0 >> 5)) : 0u;
+            const uint32_t word1_l = lane < gsz ? __ldg(bitrow_l + (pg1 >> 5)) : 0u;
             const uint32_t jb = nj % kNJ;
             if (!lwait(&sm.job_empty[jb], ((nj / kNJ) & 1u) ^ 1u)) {
                 stop = true;
@@ -357,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 J.tok[r] = r < R ? t : 0;
                 J.pos[r] = r < R ? t - cu_b : 0;
             }
-            J.word0[lane] = word0_l;
+            J.word0[0][lane] = word0_l;
+            J.word0[1][lane] = word1_l;
             if (lane == 0) {
                 J.b = b;
                 J.h = h;
@@ -365,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 J.nU = nU;
                 J.u0 = u0;
                 J.pg0 = pg0;
+                J.pg1 = pg1;
             }
             __syncwarp();
             if (lane == 0)
@@ -395,29 +452,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         phys = 0;
                     }
                 }
-                const int cnt = min(32, nU - j0);
-                for (int jj = 0; jj < cnt; ++jj, ++it) {
-                    const int ph = __shfl_sync(kFull, phys, jj);
-                    const uint32_t ks = it % kNSK, vs = it % kNSV;
-                    const int32_t row = (ph * L.Hkv + h) * 64;
-                    if (!lwait(&sm.kst_empty[ks], ((it / kNSK) & 1u) ^ 1u)) {
+                const int cnt = min(32, nU - j0); // j0 is even: a step never straddles chunks
+                for (int jj = 0; jj < cnt && !stop; jj += 2, ++stp) {
+                    const int np = min(2, cnt - jj);
+                    const int32_t row0 = (__shfl_sync(kFull, phys, jj) * L.Hkv + h) * 64;
+                    const int32_t row1 = (__shfl_sync(kFull, phys, min(jj + 1, 31)) * L.Hkv + h) * 64;
+                    // K: both pages of the step into one stage pair, on one barrier
+                    const uint32_t kp = stp % kNKP;
+                    if (!lwait(&sm.kst_empty[kp], ((stp / kNKP) & 1u) ^ 1u)) {
                         stop = true;
                         break;
                     }
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&sm.kst_full[ks], kPageBytes);
-                        tma_load_2d(sm.stage_k[ks], &tmap_k, 0, row, &sm.kst_full[ks]);
-                        sm.k_issued = it + 1;
+                        mbar_arrive_expect_tx(&sm.kst_full[kp], static_cast<uint32_t>(np) * kPageBytes);
+                        tma_load_2d(sm.stage_k[kp][0], &tmap_k, 0, row0, &sm.kst_full[kp]);
+                        if (np == 2)
+                            tma_load_2d(sm.stage_k[kp][1], &tmap_k, 0, row1, &sm.kst_full[kp]);
+                        sm.k_issued = stp + 1;
                     }
-                    if (!lwait(&sm.vst_empty[vs], ((it / kNSV) & 1u) ^ 1u)) {
-                        stop = true;
-                        break;
-                    }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&sm.vst_full[vs], kPageBytes);
-                        bulk_g2s(sm.stage_v[vs], L.V + static_cast<size_t>(row) * 128, kPageBytes,
-                                 &sm.vst_full[vs]);
-                        sm.v_issued = it + 1;
+                    // V: page by page
+                    for (int k = 0; k < np; ++k, ++it) {
+                        const uint32_t vs = it % kNSV;
+                        if (!lwait(&sm.vst_empty[vs], ((it / kNSV) & 1u) ^ 1u)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&sm.vst_full[vs], kPageBytes);
+                            bulk_g2s(sm.stage_v[vs], L.V + static_cast<size_t>(k == 0 ? row0 : row1) * 128,
+                                     kPageBytes, &sm.vst_full[vs]);
+                            sm.v_issued = it + 1;
+                        }
                     }
                     __syncwarp();
                 }
@@ -434,38 +499,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWarpMma) {
         // ---------------- MMA issue: the warp runs in lockstep, one elected lane issues ----------------
-        // Lane 0 does the waits and broadcasts the outcome, so every decision is warp-uniform;
-        // operands are computed by the converged warp (uniform registers), the elected lane
-        // (always lane 0) issues the MMAs and their commits.
+        // Every lane polls the mbarriers and a vote makes each decision warp-uniform; operands
+        // are computed by the converged warp (uniform registers), the elected lane (always
+        // lane 0) issues the MMAs and their commits.  Per step n: S_n for the step's one or two
+        // pages (N = 64 or 128), then the products of the pages of step n - 1.
         auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             const bool ok = wait_bar(bar, parity, &sm.abort_flag); // every lane polls
             return __all_sync(kFull, ok);
         };
         const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
         const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // MN-major V^T
-        uint32_t it = 0, nact = 0;
+        uint32_t it = 0, stp = 0, nact = 0;
         bool have_prev = false, ok = true;
-        PendingPV prev{};
-        auto issue_pv = [&](const PendingPV &p) -> bool {
-            const uint32_t pb = p.it & 1u;
-            if (!wwait(&sm.p_full[pb], (p.it >> 1) & 1u) || !wwait(&sm.v_full[p.vs], (p.it / kNV) & 1u))
+        // the step whose products are still to issue, kept in scalars
+        uint32_t pv_it0 = 0, pv_stp = 0, pv_np = 0, pv_nact = 0, pv_npad = 16;
+        bool pv_first = false, pv_last = false;
+        auto issue_pv = [&]() -> bool {
+            const uint32_t ob = pv_nact & 1u;
+            if (!wwait(&sm.p_full[pv_stp & 1u], (pv_stp >> 1) & 1u))
                 return false;
-            if (p.first && !wwait(&sm.o_free[p.ob], ((p.nact >> 1) & 1u) ^ 1u))
-                return false;
-            tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, static_cast<int>(2 * p.npad), true, false);
-            const uint32_t d = tmem + kColO + 128 * p.ob;
-            const uint64_t ad = desc_add(dmn, smem_u32(&sm.v[p.vs][0][0]));
-            const uint64_t bd = desc_add(dsw, smem_u32(sm.p[pb]));
-            if (elect_one()) {
+            const uint32_t idesc = idesc_bf16_f32(128, static_cast<int>(2 * pv_npad), true, false);
+            const uint32_t d = tmem + kColO + 128 * ob;
+            for (uint32_t k = 0; k < pv_np; ++k) {
+                const uint32_t page = pv_it0 + k, vs = page % kNV;
+                const bool first = pv_first && k == 0;
+                if (!wwait(&sm.v_full[vs], (page / kNV) & 1u) ||
+                    (first && !wwait(&sm.o_free[ob], ((pv_nact >> 1) & 1u) ^ 1u)))
+                    return false;
+                tc_fence_after();
+                const uint64_t ad = desc_add(dmn, smem_u32(&sm.v[vs][0][0]));
+                const uint64_t bd = desc_add(dsw, smem_u32(sm.p[pv_stp & 1u][k]));
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (p.first && kk == 0) ? 0u : 1u);
-                mma_commit(&sm.v_empty[p.vs]);
-                if (p.last)
-                    mma_commit(&sm.o_full[p.ob]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (first && kk == 0) ? 0u : 1u);
+                    mma_commit(&sm.v_empty[vs]);
+                    if (pv_last && k + 1 == pv_np)
+                        mma_commit(&sm.o_full[ob]);
+                }
+                __syncwarp();
             }
-            __syncwarp();
             return true;
         };
         for (;;) {
@@ -488,44 +561,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][0]));
             const uint64_t aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
-            for (int j = 0; j < nU; ++j, ++it) {
-                const uint32_t ks = it % kNSK, sb = it & 1u;
-                // S buffer sb was last read by the softmax of page it - 2, before it wrote the P
-                // that the product issued in the previous iteration waited for.
-                if (!wwait(&sm.kst_full[ks], (it / kNSK) & 1u)) {
+            for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
+                const uint32_t np = static_cast<uint32_t>(min(2, nU - s0));
+                const uint32_t kp = stp % kNKP, sb = stp & 1u;
+                // S buffer sb was last read by the softmax of step stp - 2, before it wrote the
+                // P that the products issued in the previous iteration waited for.
+                if (!wwait(&sm.kst_full[kp], (stp / kNKP) & 1u)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[ks]));
-                const uint32_t ds = tmem + 64 * sb;
+                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[kp][0]));
+                const uint32_t ds = tmem + kColS * sb;
+                const uint32_t idesc_s = idesc_e4m3_f32(64, static_cast<int>(64 * np));
                 if (elect_one()) {
                     // S' = q1 K^T + q2 K^T: four k-steps of 32 dims for each part
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f8_ss(ds, aq1 + 2u * kk, bk + 2u * kk, kIdescS, kk > 0 ? 1u : 0u);
+                        mma_f8_ss(ds, aq1 + 2u * kk, bk + 2u * kk, idesc_s, kk > 0 ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, kIdescS, 1u);
+                        mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, idesc_s, 1u);
                     mma_commit(&sm.s_done[sb]);
-                    mma_commit(&sm.kst_empty[ks]);
-                    if (j == nU - 1)
+                    mma_commit(&sm.kst_empty[kp]);
+                    if (s0 + static_cast<int>(np) == nU)
                         mma_commit(&sm.q_empty[qb]);
                 }
                 __syncwarp();
-                if (have_prev && !issue_pv(prev)) {
+                if (have_prev && !issue_pv()) {
                     ok = false;
                     break;
                 }
-                prev = PendingPV{it, it % kNV, nact & 1u, nact, npad, j == 0, j == nU - 1};
+                pv_it0 = it;
+                pv_stp = stp;
+                pv_np = np;
+                pv_nact = nact;
+                pv_npad = npad;
+                pv_first = s0 == 0;
+                pv_last = s0 + static_cast<int>(np) == nU;
                 have_prev = true;
+                it += np;
             }
             if (!ok)
                 break;
             ++nact;
         }
         if (ok && have_prev)
-            (void)issue_pv(prev);
+            (void)issue_pv();
     } else if (warp < kWarpSm0) {
         // ---------------- decode: Q tiles (two E4M3 parts) and E4M3 -> bf16 V tiles ----------------
         // One thread (tid 0) waits on each mbarrier; the others learn the outcome at named
@@ -605,33 +687,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kWarpEpi0) {
         // ---------------- softmax (256 threads) ----------------
         // Four threads share a row: warp (quadrant qd, half hw) reads TMEM lanes of rows
-        // 16 qd .. 16 qd + 15 and keys 32 hw .. 32 hw + 31; lane / 16 picks 16 of those keys.
-        // A row's running max m is identical in its four threads and changes only on the slow
-        // path, which runs when some element of some row exceeds its m by more than 2^8 (one
-        // OR over all 256 threads decides), so the common path needs no exchange.
+        // 16 qd .. 16 qd + 15 and, of each page, keys 32 hw .. 32 hw + 31; lane / 16 picks 16 of
+        // those keys.  A step is one or two pages.  A row's running max m is identical in its
+        // four threads and changes only on the slow path, which runs when some element of some
+        // row exceeds its m by more than 2^8 (one OR over all 256 threads decides), so the
+        // common path needs no exchange.
         const int sw = warp - kWarpSm0;     // 0..7
         const bool sleader = sw == 0 && lane == 0; // the role's one mbarrier waiter
         const int qd = sw & 3;              // TMEM lane quadrant
-        const int hw = sw >> 2;             // key half of the page read by this warp
+        const int hw = sw >> 2;             // key half of each page read by this warp
         const int row = 16 * qd + (lane & 15);
-        const int qq = 2 * hw + (lane >> 4); // 16-key quarter of the page owned by this thread
+        const int qq = 2 * hw + (lane >> 4); // 16-key quarter of each page owned by this thread
         const float crow = L.sm_scale * L.k_scale * kLog2e;
         const float acrow = fabsf(crow);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        uint32_t it = 0, nact = 0;
-        // Products known complete: [0, pv_done).  A parity wait is
-        // only unambiguous one phase ahead of what is known complete, so wait_pv steps through
-        // the phases in order.  Seeing S of page i also proves the product of page i-2 complete
-        // (S_i is issued after it).
-        // v_empty[x % kNV] completes once per product of page x; waited in page order it is
-        // unambiguous.  Lane 0 of each warp waits; the collective check that follows every
-        // call synchronises the rest.
+        uint32_t it = 0, stp = 0, nact = 0, it_prev0 = 0;
+        // Products known complete: pages [0, pv_done).  v_empty[x % kNV] completes once per
+        // product of page x, and a parity wait is only unambiguous one phase ahead of what is
+        // known complete, so wait_pv steps through the phases in page order.  Seeing S of step
+        // n also proves the products of step n - 2 complete (they were issued before it).  Only
+        // the leader waits (every thread advances pv_done alike); the collective vote that
+        // follows every call passes the outcome on.
         uint32_t pv_done = 0;
         auto wait_pv = [&](uint32_t x) -> bool { // product of page x complete
             for (; pv_done <= x; ++pv_done)
                 if (sleader && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
                     return false;
             return true;
+        };
+        auto allowed = [&](int pg, uint32_t word, int pos, int own) -> int { // keys of page pg in my quarter
+            int n_allow = 0;
+            if ((word >> (pg & 31)) & 1u)
+                n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
+            return min(max(n_allow - 16 * qq, 0), 16);
         };
         bool ok = true;
         for (;;) {
@@ -660,56 +748,62 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain factor
             const float inv = exp2i(-J.qexp[row]);
             const float crow_r = crow * inv, acrow_r = acrow * inv;
-            int pg_next = J.pg0;
-            uint32_t word_next = valid ? J.word0[row / L.G] : 0u;
+            int pg_a = J.pg0, pg_b = J.pg1;
+            uint32_t word_a = valid ? J.word0[0][row / L.G] : 0u;
+            uint32_t word_b = valid ? J.word0[1][row / L.G] : 0u;
             warp_arrive(&sm.job_empty[jb], lane);
             const uint32_t ob = nact & 1u;
             const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
             float m_used = -INFINITY, l_part = 0.f;
-            for (int j = 0; j < nU; ++j, ++it) {
-                const int pg = pg_next;
-                const uint32_t word = word_next;
-                if (j + 1 < nU) { // next page's id and my membership word, fetched early
-                    pg_next = L.union_pages[u0 + j + 1];
-                    word_next = valid ? __ldg(bitrow + (pg_next >> 5)) : 0u;
+            for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
+                const int np = min(2, nU - s0);
+                const int pgA = pg_a, pgB = pg_b;
+                const uint32_t wA = word_a, wB = word_b;
+                // the next step's page ids and my membership words, fetched early
+                if (s0 + 2 < nU) {
+                    pg_a = L.union_pages[u0 + s0 + 2];
+                    word_a = valid ? __ldg(bitrow + (pg_a >> 5)) : 0u;
                 }
-                const uint32_t sb = it & 1u, pb = it & 1u;
+                if (s0 + 3 < nU) {
+                    pg_b = L.union_pages[u0 + s0 + 3];
+                    word_b = valid ? __ldg(bitrow + (pg_b >> 5)) : 0u;
+                }
+                const uint32_t sb = stp & 1u;
+                const uint32_t it0 = it;
                 // every abort decision of this role is collective: a thread that left alone
                 // would strand the others at the named barrier or in a warp-wide TMEM load
-                ok = !sleader || wait_bar(&sm.s_done[sb], (it >> 1) & 1u, &sm.abort_flag);
+                ok = !sleader || wait_bar(&sm.s_done[sb], (stp >> 1) & 1u, &sm.abort_flag);
                 if (softmax_bar_or(!ok)) {
                     ok = false;
                     break;
                 }
-                if (it >= 2 && pv_done < it - 1)
-                    pv_done = it - 1;
+                if (pv_done < it_prev0)
+                    pv_done = it_prev0;
+                // S of the step is read twice (for the max, then for P), one page at a time, so
+                // that only sixteen scores are live in registers.
                 tc_fence_after();
-                uint32_t sv[16];
-                tmem_ld_16x32bx2_x16(tmem + lane_base + 64 * sb + 32 * hw, sv);
-                tmem_ld_wait16(sv);
-                tc_fence_before();
-
-                int n_allow = 0;
-                if ((word >> (pg & 31)) & 1u)
-                    n_allow = pg < own ? 64 : (pg == own ? (pos & 63) + 1 : 0);
-                const int nq = min(max(n_allow - 16 * qq, 0), 16); // allowed keys in my quarter
-                float lm = -INFINITY;
-                if (crow >= 0.f) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (e < nq)
-                            lm = fmaxf(lm, __uint_as_float(sv[e]));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (e < nq)
-                            lm = fmaxf(lm, -__uint_as_float(sv[e]));
+                const uint32_t s_addr = tmem + lane_base + kColS * sb + 32 * hw;
+                const int nqA = allowed(pgA, wA, pos, own);
+                const int nqB = np == 2 ? allowed(pgB, wB, pos, own) : 0;
+                const bool flip = crow < 0.f;
+                float lm;
+                {
+                    uint32_t sv[16];
+                    tmem_ld_16x32bx2_x16(s_addr, sv);
+                    tmem_ld_wait16(sv);
+                    lm = quarter_max(sv, nqA, flip);
+                    if (np == 2) {
+                        tmem_ld_16x32bx2_x16(s_addr + 64, sv);
+                        tmem_ld_wait16(sv);
+                        lm = fmaxf(lm, quarter_max(sv, nqB, flip));
+                    }
                 }
-                if (nq > 0)
+                const bool any = nqA > 0 || nqB > 0;
+                if (any)
                     lm *= acrow_r;
-                if (softmax_bar_or(nq > 0 && lm > m_used + kRescaleLog2)) {
+                if (softmax_bar_or(any && lm > m_used + kRescaleLog2)) {
                     // slow path: the row's four threads agree on its max
-                    sm.qmax[row][qq] = lm;
+                    sm.qmax[row][qq] = any ? lm : -INFINITY;
                     softmax_bar();
                     const float M = fmaxf(fmaxf(sm.qmax[row][0], sm.qmax[row][1]),
                                           fmaxf(sm.qmax[row][2], sm.qmax[row][3]));
@@ -724,11 +818,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         m_used = M;
                     }
                     if (qq == 0)
-                        sm.alpha[pb][row] = rescale ? alpha : 1.f;
+                        sm.alpha[sb][row] = rescale ? alpha : 1.f;
                     if (softmax_bar_or(rescale)) {
-                        // O^T[d, r] *= alpha[r] for both accumulator halves, after the previous
-                        // page's product (the only one that may still run).
-                        ok = j == 0 || wait_pv(it - 1);
+                        // O^T[d, r] *= alpha[r] for both accumulator halves, once every product
+                        // issued so far (those of the pages before this step) has completed.
+                        ok = s0 == 0 || wait_pv(it0 - 1);
                         if (softmax_bar_or(!ok)) {
                             ok = false;
                             break;
@@ -741,48 +835,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int r0 = c0 < npad ? c0 : c0 - npad;
 #pragma unroll
                             for (int e = 0; e < 16; ++e)
-                                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[pb][r0 + e]);
+                                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[sb][r0 + e]);
                             tmem_st16(o_addr + c0, o);
                         }
                         tmem_st_wait();
                     }
                 }
                 const float negm = m_used == -INFINITY ? 0.f : -m_used;
-                // P buffer pb was last read by the product of page it-2, complete since
-                // S of page it (issued after it) is.  Rows 0..npad-1 hold P_hi, rows
-                // npad..2 npad-1 P_lo; only rows < npad write.
-                uint8_t *phi = sm.p[pb], *plo = sm.p[pb] + npad * 128;
-                uint32_t hi[8], lo[8];
-                if (__all_sync(kFull, nq == 16)) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), crow_r, negm));
-                        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow_r, negm));
-                        l_part += p0 + p1;
-                        split_pair(p0, p1, hi[e], lo[e]);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), crow_r, negm)) : 0.f;
-                        const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), crow_r, negm)) : 0.f;
-                        l_part += p0 + p1;
-                        split_pair(p0, p1, hi[e], lo[e]);
-                    }
+                // P buffers [sb][*] were last read by the products of step stp - 2, complete
+                // since S of this step (issued after them) is.
+                for (int k = 0; k < np; ++k) {
+                    uint32_t sv[16];
+                    tc_fence_after();
+                    tmem_ld_16x32bx2_x16(s_addr + 64 * k, sv);
+                    tmem_ld_wait16(sv);
+                    l_part += emit_p(sv, k == 0 ? nqA : nqB, crow_r, negm, sm.p[sb][k], row, qq, npad);
                 }
-                if (row < npad) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint32_t o = swz(row, 2 * qq + c);
-                        *reinterpret_cast<uint4 *>(phi + o) =
-                            make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                        *reinterpret_cast<uint4 *>(plo + o) =
-                            make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-                    }
-                }
+                tc_fence_before();
                 fence_proxy_async_smem();
                 tc_fence_before();
-                warp_arrive(&sm.p_full[pb], lane);
+                warp_arrive(&sm.p_full[sb], lane);
+                it_prev0 = it0;
+                it += np;
             }
             if (!ok)
                 break;
@@ -869,9 +943,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the last copy issued on each stage, and every product issued so far.
         if (tid == 0) {
             const uint32_t nk = sm.k_issued, nv = sm.v_issued;
-            for (uint32_t s = 0; s < kNSK && s < nk; ++s) {
-                const uint32_t last = s + ((nk - 1 - s) / kNSK) * kNSK;
-                (void)mbar_wait(&sm.kst_full[s], (last / kNSK) & 1u);
+            for (uint32_t s = 0; s < kNKP && s < nk; ++s) {
+                const uint32_t last = s + ((nk - 1 - s) / kNKP) * kNKP;
+                (void)mbar_wait(&sm.kst_full[s], (last / kNKP) & 1u);
             }
             for (uint32_t s = 0; s < kNSV && s < nv; ++s) {
                 const uint32_t last = s + ((nv - 1 - s) / kNSV) * kNSV;
