@@ -33,7 +33,7 @@ METRIC = "complete-call ms and useful TFLOP/s (grouping incl.) at 1 B200; % of r
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=4)
@@ -121,26 +121,36 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    """nvidia-smi samples every 20 ms, started before the warm-up (its start-up takes longer
+    than a short timed region) and reduced to the samples taken inside the timed window."""
+
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host monotonic time, csv line)
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.monotonic() + 5.0
+            while not self.lines and time.monotonic() < deadline:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -153,7 +163,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.window is not None:
+            inside = [x for x in lines if self.window[0] <= x[0] <= self.window[1]]
+            lines = inside if inside else lines
+        for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -301,6 +315,7 @@ def run_ours(args):
         api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
                     groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=O, status=status)
 
+    clocks = ClockSampler(dev.index).__enter__()
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()
@@ -317,17 +332,19 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], args.W, args.g,
-                         groups=groups, status=status)
-            ev[i][1].record(stream)
-            api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
-                        groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=O, status=status)
-            ev[i][2].record(stream)
-        torch.cuda.synchronize()
+    t_start = time.monotonic()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], args.W, args.g,
+                     groups=groups, status=status)
+        ev[i][1].record(stream)
+        api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
+                    groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=O, status=status)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(t_start, time.monotonic())
+    clocks.__exit__(None, None, None)
     if world > 1:
         dist.barrier()
     api.check_status(status, "bench timed region")
@@ -391,7 +408,9 @@ def run_ours(args):
     attn_mean = statistics.mean(attn_ms)
     achieved = union_bytes / (attn_mean * 1e-3) / 1e9
     ksrc = os.path.join(ROOT, "dynamic_sparse_attention_pw_b200", "csrc")
-    khash = source_hash(os.path.join(ksrc, "pw_attn.cu"), os.path.join(ksrc, "pw_sm100.cuh"))
+    khash = source_hash(*(os.path.join(ksrc, f) for f in
+                          ("pw_attn.cu", "pw_attn_ws.cu", "pw_attn_common.cuh", "pw_sm100.cuh")))
+    kname = "k_union_attn_ws" if args.g * wl.G <= 64 else "k_union_attn"
     roof_ms = max(union_bytes / (hbm * 1e9), exec_flops / (bf16 * 1e12)) * 1e3
     line = {
         "metric": METRIC,
@@ -404,13 +423,13 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16 operands / fp32 accumulate (E4M3 KV, bf16 Q/O)",
+        "dtype": "e4m3 x e4m3 (S, Q split exactly in two e4m3 parts) and bf16 x bf16 (PV), fp32 accumulate",
         "data": "synthetic",
         "config": config_of(wl, args),
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic_from_profile(khash),
-            "kernel": "k_union_attn", "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"
+            "kernel": kname, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"
             if src == "measured" else "fallback 6650 GB/s",
             "algorithmic_bytes_per_launch": union_bytes,
             "kernel_ms": attn_mean,
