@@ -156,3 +156,17 @@ def test_frequent_rescales(scale):
     got, _ = _run(inp, 64, 8)
     parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128),
                         f"scale {scale}")
+
+
+def test_q_rows_with_wide_dynamic_range():
+    # Q elements spread over 18 binades within every row, so part of each row lies below 2^-9
+    # of the row's largest, where the kernel's two-part E4M3 form of Q is not exact; the
+    # scores still depend on those elements.
+    wl = _small(15, [640, 200], 8, 2, 6, shuffled_pages=True)
+    inp = dict(parity.inputs(wl))
+    q = torch.from_numpy(inp["Q"].view(np.int16)).view(torch.bfloat16).float()
+    gen = torch.Generator().manual_seed(15)
+    q = q * torch.pow(2.0, torch.randint(-14, 4, q.shape, generator=gen).float())
+    inp["Q"] = q.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got, _ = _run(inp, 32, 8)
+    parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128), "wide Q rows")
