@@ -252,6 +252,18 @@ __device__ __forceinline__ void split_q8(const uint4 v, float scale, uint2 &q1, 
 __device__ __forceinline__ float quarter_max(const uint32_t (&sv)[16], int nq, bool flip)
 {
     float lm = -INFINITY;
+    if (__all_sync(0xFFFFFFFFu, nq == 16)) { // every key allowed: a tree, no predicates
+        float m[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            m[e] = flip ? -__uint_as_float(sv[e]) : __uint_as_float(sv[e]);
+#pragma unroll
+        for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e)
+                m[e] = fmaxf(m[e], m[e + w]);
+        return m[0];
+    }
     if (!flip) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
