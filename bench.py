@@ -345,6 +345,14 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks.mark(t_start, time.monotonic())
     clocks.__exit__(None, None, None)
+    # secondary figure: the same calls with L2 left warm (no flush between them)
+    wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(K, 10))]
+    for e in wev:
+        e[0].record(stream)
+        step()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    warm_ms = [e[0].elapsed_time(e[1]) for e in wev]
     if world > 1:
         dist.barrier()
     api.check_status(status, "bench timed region")
@@ -436,6 +444,9 @@ def run_ours(args):
         },
         "breakdown": {
             "group_ms": statistics.mean(group_ms), "attn_ms": attn_mean,
+            "group_ms_median": statistics.median(group_ms), "attn_ms_median": statistics.median(attn_ms),
+            "complete_call_ms_median": statistics.median(step_ms),
+            "complete_call_ms_warm_l2_median": statistics.median(warm_ms),
             "complete_call_ms": ms_per_step,
             "roofline_ms": roof_ms, "complete_call_frac_of_roofline": roof_ms / ms_per_step,
             "attn_frac_of_roofline": roof_ms / attn_mean,
