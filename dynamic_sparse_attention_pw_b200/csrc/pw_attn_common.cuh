@@ -1,5 +1,6 @@
 // pw_attn_common.cuh -- device helpers shared by the union-attention kernels: operand-tile
-// swizzle, exact E4M3 -> bf16 decode with integer bit operations, the bf16 hi/lo split of P.
+// swizzle, exact E4M3 -> bf16 (integer bit operations) and E4M3 -> f16 (hardware cvt) decodes,
+// the bf16 and f16 hi/lo splits of P.
 #pragma once
 
 #include <cstdint>
@@ -73,6 +74,52 @@ __device__ __forceinline__ void decode_page(const uint8_t *src, uint8_t (*dst)[6
             *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
         }
     }
+}
+
+// 64 keys x 128 dims E4M3 (row-major) -> two swizzled 64-dim f16 blocks, the same tile layout
+// as decode_page.  E4M3 values are exact in f16 (subnormals included); the hardware converts
+// two codes per instruction.
+template <int NT>
+__device__ __forceinline__ void decode_page_f16(const uint8_t *src, uint8_t (*dst)[64 * 128], int tid)
+{
+#pragma unroll
+    for (int rep = 0; rep < 512 / NT; ++rep) {
+        const int q = tid + NT * rep;
+        const int key = q >> 3, c16 = q & 7;
+        const uint4 x = *reinterpret_cast<const uint4 *>(src + key * 128 + c16 * 16);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
+                "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, u;\n\t}\n"
+                : "=r"(h[2 * i]), "=r"(h[2 * i + 1])
+                : "r"(w[i]));
+        const uint4 h0 = make_uint4(h[0], h[1], h[2], h[3]), h1 = make_uint4(h[4], h[5], h[6], h[7]);
+        uint8_t *blk = dst[c16 >> 2];
+        const int j0 = (2 * c16) & 7;
+        if (c16 < 4) {
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
+        } else {
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0 + 1)) = h1;
+            *reinterpret_cast<uint4 *>(blk + swz(key, j0)) = h0;
+        }
+    }
+}
+
+// p -> (hi, lo) f16 halves of two packed words: hi = p rounded to f16, lo = p - hi rounded to
+// f16 (p - hi is exact in f32).  For p in [2^-3, 256] the pair carries about 22 significant
+// bits; below, the absolute error stays under 2^-25.
+__device__ __forceinline__ void split_pair_f16(float p0, float p1, uint32_t &hi2, uint32_t &lo2)
+{
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hi2) : "f"(p1), "f"(p0));
+    float h0, h1;
+    asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}\n"
+        : "=f"(h0), "=f"(h1)
+        : "r"(hi2));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo2) : "f"(p1 - h1), "f"(p0 - h0));
 }
 
 __device__ __forceinline__ float ex2(float x)

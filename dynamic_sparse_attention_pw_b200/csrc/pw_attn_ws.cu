@@ -9,11 +9,12 @@
 // is scaled by a power of two and split into two E4M3 parts, q' = q1 + q2, which is exact for
 // every element within 2^9 of the row's largest (an 8-bit bf16 significand is a 4-bit E4M3
 // significand plus a remainder of at most 4 bits); S = (q1 K^T + q2 K^T) 2^-s.  The product
-// O^T = V^T P^T stays on bf16 operands (V decoded exactly, P split into bf16 hi + lo parts).
+// O^T = V^T P^T runs on f16 operands: V decoded exactly (E4M3 is a subset of f16), P split
+// into f16 hi + lo parts.
 //
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
 //   warps 0-3    decode   Q tile of each group (gathered by query ID, scaled, split into two
-//                         E4M3 parts); E4M3 V pages -> bf16 operand tiles
+//                         E4M3 parts); E4M3 V pages -> f16 operand tiles
 //   warps 4-11   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
 //                         O^T rescale, per-row sums of each group
 //   warps 12-15  epilogue O^T of a finished group -> bf16 rows of O (one warp per TMEM lane
@@ -25,7 +26,7 @@
 // its scheduler delays its waits and issues.
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
 // (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, which the
-// epilogue adds.  A K stage is free once S is done, a V stage once it is decoded, a bf16 V slot
+// epilogue adds.  A K stage is free once S is done, a V stage once it is decoded, an f16 V slot
 // once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
 // mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
 // other roles.
@@ -47,7 +48,7 @@ using namespace attn;
 constexpr int kNKP = 2;       // E4M3 K stage pairs (one S step each)
 constexpr int kNSV = 3;       // E4M3 V page stages
 constexpr int kNJ = 3;        // group records in flight
-constexpr int kNV = 3;        // bf16 V slots
+constexpr int kNV = 3;        // f16 V slots
 constexpr int kDecThreads = 128;
 constexpr int kSmThreads = 256;
 constexpr int kEpiThreads = 128;
@@ -73,7 +74,7 @@ struct GroupJob {
 
 struct __align__(1024) WsSmem {
     uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
-    uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] bf16, swizzled
+    uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] f16, swizzled
     // [step parity][page of the step][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
     uint8_t p[2][2][128 * 128];
     // E4M3 K pages, 128-byte swizzled by the tensor copy; the two pages of a step sit in one
@@ -291,7 +292,7 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
             const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm));
             sum += p0 + p1;
-            split_pair(p0, p1, hi[e], lo[e]);
+            split_pair_f16(p0, p1, hi[e], lo[e]);
         }
     } else {
 #pragma unroll
@@ -299,7 +300,7 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm)) : 0.f;
             const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm)) : 0.f;
             sum += p0 + p1;
-            split_pair(p0, p1, hi[e], lo[e]);
+            split_pair_f16(p0, p1, hi[e], lo[e]);
         }
     }
     if (row < npad) {
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ob = pv_nact & 1u;
             if (!wwait(&sm.p_full[pv_stp & 1u], (pv_stp >> 1) & 1u))
                 return false;
-            const uint32_t idesc = idesc_bf16_f32(128, static_cast<int>(2 * pv_npad), true, false);
+            const uint32_t idesc = idesc_f16_f32(128, static_cast<int>(2 * pv_npad), true, false);
             const uint32_t d = tmem + kColO + 128 * ob;
             for (uint32_t k = 0; k < pv_np; ++k) {
                 const uint32_t page = pv_it0 + k, vs = page % kNV;
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && have_prev)
             (void)issue_pv();
     } else if (warp < kWarpSm0) {
-        // ---------------- decode: Q tiles (two E4M3 parts) and E4M3 -> bf16 V tiles ----------------
+        // ---------------- decode: Q tiles (two E4M3 parts) and E4M3 -> f16 V tiles ----------------
         // One thread (tid 0) waits on each mbarrier; the others learn the outcome at named
         // barrier kBarDecode.
         uint32_t it = 0, nact = 0;
@@ -684,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                decode_page<kDecThreads>(sm.stage_v[st], sm.v[vs], tid);
+                decode_page_f16<kDecThreads>(sm.stage_v[st], sm.v[vs], tid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
