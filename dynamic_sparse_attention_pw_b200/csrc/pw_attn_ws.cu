@@ -13,15 +13,17 @@
 // into f16 hi + lo parts.
 //
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
-//   warps 0-3    decode   Q tile of each group (gathered by query ID, scaled, split into two
-//                         E4M3 parts); E4M3 V pages -> f16 operand tiles
-//   warps 4-11   softmax  S -> P for each page (four threads per row, 16 keys each), lazy
-//                         O^T rescale, per-row sums of each group
-//   warps 12-15  epilogue O^T of a finished group -> bf16 rows of O (one warp per TMEM lane
-//                         quadrant), while the softmax warps already work on the next group
-//   warp 16      load     TMA copies of the union pages: K through a tensor map with the
-//                         128-byte swizzle the MMA reads, V as plain bulk copies
-//   warp 17      MMA      S_i = Q K_i^T issued one page ahead of O^T += V_{i-1}^T P_{i-1}^T
+//   warps 0-3    decode   E4M3 V pages -> f16 operand tiles
+//   warps 4-11   softmax  S -> P for each step of one or two pages (four threads per row,
+//                         16 keys of each page each), lazy O^T rescale, per-row sums of each group
+//   warps 12-15  epilogue Q tile of the next group (scaled, split into two E4M3 parts) while
+//                         the current one runs, then O^T of the finished group -> bf16 rows of O
+//                         (one warp per TMEM lane quadrant)
+//   warp 16      load     one group ahead: group records (rows, positions, first membership
+//                         words), the next group's Q rows by TMA, and the union pages: K through
+//                         a tensor map with the 128-byte swizzle the MMA reads, V by bulk copy
+//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O^T += V^T P^T for
+//                         the pages of step n - 1
 // Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
 // its scheduler delays its waits and issues.
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
@@ -337,10 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Arrivals from the decode and softmax roles are one per warp (after __syncwarp).
         for (int s = 0; s < kNJ; ++s) {
             mbar_init(&sm.job_full[s], 1);
-            mbar_init(&sm.job_empty[s], kDecThreads / 32 + 1 + kSmThreads / 32);
+            mbar_init(&sm.job_empty[s], kDecThreads / 32 + 1 + kSmThreads / 32 + kEpiThreads / 32);
         }
         mbar_init(&sm.qraw_full, 1);
-        mbar_init(&sm.qraw_empty, kDecThreads / 32);
+        mbar_init(&sm.qraw_empty, kEpiThreads / 32);
         for (int s = 0; s < kNKP; ++s) {
             mbar_init(&sm.kst_full[s], 1);
             mbar_init(&sm.kst_empty[s], 1);
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_done[s], 1);
             mbar_init(&sm.p_full[s], kSmThreads / 32);
-            mbar_init(&sm.q_full[s], kDecThreads / 32);
+            mbar_init(&sm.q_full[s], kEpiThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
             mbar_init(&sm.o_full[s], 1);
             mbar_init(&sm.l_full[s], kSmThreads / 32);
@@ -381,80 +383,121 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kWarpLoad) {
         // ---------------- load: group records, Q rows, union pages -> stages ----------------
-        // Runs pages ahead of the other roles, so the latency of its dependent global loads
-        // (group -> query IDs -> positions and membership words) stays off their path.  Every
-        // lane polls its mbarriers; lane 0 issues the page copies.
+        // Works one group ahead: while it issues the pages of group n it has already published
+        // the record of group n + 1, and it copies group n + 1's Q rows as soon as the raw Q
+        // buffer is free (the epilogue warps then prepare that Q tile in the middle of group n).
+        // The latency of its dependent global loads (group -> query IDs -> positions and
+        // membership words) stays off the other roles' path.  Every lane polls its mbarriers;
+        // lane 0 issues the copies.
         auto lwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             return __all_sync(kFull, wait_bar(bar, parity, &sm.abort_flag));
         };
-        uint32_t it = 0, stp = 0, nj = 0;
-        bool stop = false;
-        for (int64_t gi = g0; gi < L.n_groups && !stop; gi += gstep) {
-            const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
-            const int gsz = L.gsize[gi], R = gsz * L.G;
-            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
-            if (nU == 0) {
-                // no union page: every row of the group is empty
-                for (int idx = lane; idx < R * 16; idx += 32) {
-                    const int r = idx >> 4, c = idx & 15, mi = r / L.G;
-                    const int64_t tok = L.qids[gi * L.g + mi];
-                    const int hq = h * L.G + (r - mi * L.G);
-                    reinterpret_cast<uint4 *>(L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim)[c] =
-                        make_uint4(0u, 0u, 0u, 0u);
+        struct GMeta {
+            int64_t gi;
+            int b, h, gsz, R, u0, nU, pg0, pg1;
+            int32_t tok_l, cu_b;   // lane l: query l of the group
+            uint32_t w0_l, w1_l;   // lane l: its membership words of the first two union pages
+        };
+        // The next group with union pages, from gi on; groups without any get their zero rows.
+        auto next_group = [&](int64_t gi, GMeta &m) -> bool {
+            for (; gi < L.n_groups; gi += gstep) {
+                const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
+                const int gsz = L.gsize[gi], R = gsz * L.G;
+                const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
+                if (nU == 0) {
+                    for (int idx = lane; idx < R * 16; idx += 32) {
+                        const int r = idx >> 4, c = idx & 15, mi = r / L.G;
+                        const int64_t tok = L.qids[gi * L.g + mi];
+                        const int hq = h * L.G + (r - mi * L.G);
+                        reinterpret_cast<uint4 *>(L.O + (static_cast<size_t>(tok) * L.Hq + hq) * kHeadDim)[c] =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    continue;
                 }
-                continue;
+                m.gi = gi;
+                m.b = b;
+                m.h = h;
+                m.gsz = gsz;
+                m.R = R;
+                m.u0 = u0;
+                m.nU = nU;
+                m.tok_l = lane < gsz ? L.qids[gi * L.g + lane] : 0;
+                m.cu_b = L.cu[b];
+                m.pg0 = L.union_pages[u0];
+                m.pg1 = nU > 1 ? L.union_pages[u0 + 1] : m.pg0;
+                const uint32_t *bitrow = L.bits + (static_cast<size_t>(m.tok_l) * L.Hkv + h) * L.words;
+                m.w0_l = lane < gsz ? __ldg(bitrow + (m.pg0 >> 5)) : 0u;
+                m.w1_l = lane < gsz ? __ldg(bitrow + (m.pg1 >> 5)) : 0u;
+                return true;
             }
-            // the group record
-            const int32_t tok_l = lane < gsz ? L.qids[gi * L.g + lane] : 0;
-            const int32_t cu_b = L.cu[b];
-            const int pg0 = L.union_pages[u0], pg1 = nU > 1 ? L.union_pages[u0 + 1] : pg0;
-            const uint32_t *bitrow_l = L.bits + (static_cast<size_t>(tok_l) * L.Hkv + h) * L.words;
-            const uint32_t word0_l = lane < gsz ? __ldg(bitrow_l + (pg0 >> 5)) : 0u;
-            const uint32_t word1_l = lane < gsz ? __ldg(bitrow_l + (pg1 >> 5)) : 0u;
-            const uint32_t jb = nj % kNJ;
-            if (!lwait(&sm.job_empty[jb], ((nj / kNJ) & 1u) ^ 1u)) {
-                stop = true;
-                break;
-            }
+            return false;
+        };
+        // Record of job n (or the end marker when m is null) into its ring slot.
+        auto publish = [&](uint32_t n, const GMeta *m) -> bool {
+            const uint32_t jb = n % kNJ;
+            if (!lwait(&sm.job_empty[jb], ((n / kNJ) & 1u) ^ 1u))
+                return false;
             GroupJob &J = sm.job[jb];
+            if (m != nullptr) {
 #pragma unroll
-            for (int r0 = 0; r0 < 64; r0 += 32) {
-                const int r = r0 + lane;
-                const int mi = min(r / L.G, 31);
-                const int32_t t = __shfl_sync(kFull, tok_l, mi);
-                J.tok[r] = r < R ? t : 0;
-                J.pos[r] = r < R ? t - cu_b : 0;
+                for (int r0 = 0; r0 < 64; r0 += 32) {
+                    const int r = r0 + lane;
+                    const int mi = min(r / L.G, 31);
+                    const int32_t t = __shfl_sync(kFull, m->tok_l, mi);
+                    J.tok[r] = r < m->R ? t : 0;
+                    J.pos[r] = r < m->R ? t - m->cu_b : 0;
+                }
+                J.word0[0][lane] = m->w0_l;
+                J.word0[1][lane] = m->w1_l;
             }
-            J.word0[0][lane] = word0_l;
-            J.word0[1][lane] = word1_l;
             if (lane == 0) {
-                J.b = b;
-                J.h = h;
-                J.R = R;
-                J.nU = nU;
-                J.u0 = u0;
-                J.pg0 = pg0;
-                J.pg1 = pg1;
+                J.nU = m != nullptr ? m->nU : -1;
+                if (m != nullptr) {
+                    J.b = m->b;
+                    J.h = m->h;
+                    J.R = m->R;
+                    J.u0 = m->u0;
+                    J.pg0 = m->pg0;
+                    J.pg1 = m->pg1;
+                }
             }
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sm.job_full[jb]);
-            // the group's Q rows: query qi's G heads are G consecutive rows of Q
-            if (!lwait(&sm.qraw_empty, (nj & 1u) ^ 1u)) {
+            return true;
+        };
+        // Q rows of job n: query qi's G heads are G consecutive rows of Q.  The raw buffer is
+        // free (the caller waited for it).
+        auto copy_q = [&](uint32_t n, const GMeta &m) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.qraw_full, static_cast<uint32_t>(m.R) * 256u);
+                sm.q_issued = n + 1;
+            }
+            __syncwarp();
+            if (lane < m.gsz)
+                bulk_g2s(sm.q_raw + lane * L.G * 256,
+                         L.Q + (static_cast<size_t>(m.tok_l) * L.Hq + m.h * L.G) * kHeadDim,
+                         static_cast<uint32_t>(L.G) * 256u, &sm.qraw_full);
+        };
+        uint32_t it = 0, stp = 0, nj = 0;
+        bool stop = false;
+        GMeta cur{}, nxt{};
+        bool has_cur = next_group(g0, cur);
+        if (has_cur)
+            stop = !publish(0, &cur) || !lwait(&sm.qraw_empty, 1u);
+        else
+            stop = !publish(0, nullptr);
+        if (has_cur && !stop)
+            copy_q(0, cur);
+        while (has_cur && !stop) {
+            const bool has_nxt = next_group(cur.gi + gstep, nxt);
+            if (!publish(nj + 1, has_nxt ? &nxt : nullptr)) {
                 stop = true;
                 break;
             }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.qraw_full, static_cast<uint32_t>(R) * 256u);
-                sm.q_issued = nj + 1;
-            }
-            __syncwarp();
-            if (lane < gsz)
-                bulk_g2s(sm.q_raw + lane * L.G * 256,
-                         L.Q + (static_cast<size_t>(tok_l) * L.Hq + h * L.G) * kHeadDim,
-                         static_cast<uint32_t>(L.G) * 256u, &sm.qraw_full);
-            ++nj;
-            // the union pages
+            bool q_pending = has_nxt; // Q rows of job nj + 1, once job nj's raw rows are used
+            const uint32_t q_parity = (nj & 1u); // phase nj of qraw_empty (released by job nj's split)
+            const int b = cur.b, h = cur.h, u0 = cur.u0, nU = cur.nU;
             for (int j0 = 0; j0 < nU && !stop; j0 += 32) {
                 int phys = 0;
                 if (j0 + lane < nU) {
@@ -498,17 +541,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     __syncwarp();
+                    // the next job's Q rows, as soon as the raw buffer is free (no wait here)
+                    if (!stop && q_pending && __all_sync(kFull, mbar_try_wait(&sm.qraw_empty, q_parity))) {
+                        copy_q(nj + 1, nxt);
+                        q_pending = false;
+                    }
                 }
             }
-        }
-        if (!stop) { // end marker
-            const uint32_t jb = nj % kNJ;
-            if (lwait(&sm.job_empty[jb], ((nj / kNJ) & 1u) ^ 1u)) {
-                if (lane == 0) {
-                    sm.job[jb].nU = -1;
-                    mbar_arrive(&sm.job_full[jb]);
+            if (!stop && q_pending) {
+                if (!lwait(&sm.qraw_empty, q_parity)) {
+                    stop = true;
+                    break;
                 }
+                copy_q(nj + 1, nxt);
             }
+            cur = nxt;
+            has_cur = has_nxt;
+            ++nj;
         }
     } else if (warp == kWarpMma) {
         // ---------------- MMA issue: the warp runs in lockstep, one elected lane issues ----------------
@@ -622,59 +671,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && have_prev)
             (void)issue_pv();
     } else if (warp < kWarpSm0) {
-        // ---------------- decode: Q tiles (two E4M3 parts) and E4M3 -> f16 V tiles ----------------
+        // ---------------- decode: E4M3 -> f16 V tiles ----------------
         // One thread (tid 0) waits on each mbarrier; the others learn the outcome at named
         // barrier kBarDecode.
         uint32_t it = 0, nact = 0;
         bool ok = true;
         for (;;) {
-            const uint32_t jb = nact % kNJ, qb = nact & 1u;
+            const uint32_t jb = nact % kNJ;
             if (!role_wait(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag, tid == 0, kBarDecode,
                            kDecThreads)) {
                 ok = false;
                 break;
             }
-            GroupJob &J = sm.job[jb];
-            const int R = J.R, nU = J.nU;
-            if (nU < 0) {
-                warp_arrive(&sm.job_empty[jb], lane);
-                break;
-            }
-            // Q tile buffer qb was last read by the last S of group nact - 2; the raw rows of
-            // this group have landed.
-            bool got = true;
-            if (tid == 0)
-                got = wait_bar(&sm.q_empty[qb], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag) &&
-                      wait_bar(&sm.qraw_full, nact & 1u, &sm.abort_flag);
-            if (bar_or(kBarDecode, kDecThreads, !got)) {
-                ok = false;
-                break;
-            }
-            // Row r of the tile is query head h G + r % G of query r / G.  Sixteen consecutive
-            // lanes hold one row (eight dims each) and agree on its scale.
-#pragma unroll
-            for (int rep = 0; rep < 1024 / kDecThreads; ++rep) {
-                const int qn = tid + kDecThreads * rep;
-                const int row = qn >> 4, c = qn & 15;
-                const uint4 val = row < R ? *reinterpret_cast<const uint4 *>(sm.q_raw + row * 256 + c * 16)
-                                          : make_uint4(0u, 0u, 0u, 0u);
-                uint32_t e = max_exp8(val);
-#pragma unroll
-                for (int o = 8; o > 0; o >>= 1)
-                    e = max(e, __shfl_xor_sync(kFull, e, o));
-                const int sexp = q_scale_exp(e);
-                uint2 q1, q2;
-                split_q8(val, exp2i(sexp), q1, q2);
-                const uint32_t off = swz(row, c >> 1) + 8u * (c & 1);
-                *reinterpret_cast<uint2 *>(sm.q[qb][0] + off) = q1;
-                *reinterpret_cast<uint2 *>(sm.q[qb][1] + off) = q2;
-                if (c == 0)
-                    J.qexp[row] = sexp;
-            }
-            fence_proxy_async_smem();
-            warp_arrive(&sm.q_full[qb], lane);
-            warp_arrive(&sm.qraw_empty, lane);
+            const int nU = sm.job[jb].nU;
             warp_arrive(&sm.job_empty[jb], lane);
+            if (nU < 0)
+                break;
             for (int j = 0; j < nU; ++j, ++it) {
                 const uint32_t st = it % kNSV, vs = it % kNV;
                 bool got = true;
@@ -885,28 +897,82 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++nact;
         }
     } else {
-        // ---------------- epilogue (128 threads) ----------------
-        // Warp e reads TMEM lane quadrant e: thread (e, lane) holds head dimension 32 e + lane of
-        // every row, so each row's 32 dimensions leave as one 64-byte store per warp.  Row
-        // metadata (output row index, 1 / l) is computed lane-parallel, 32 rows at a time, and
-        // broadcast with shuffles; no barrier spans the four warps, so each leaves on its own
-        // when a wait gives up.
+        // ---------------- epilogue (128 threads): Q tiles, and O of finished groups ----------------
+        // Per group n: first the Q tile of group n + 1 (its raw rows land while group n runs; the
+        // split into two E4M3 parts is off every other role's path here), then the output of
+        // group n once its last product is done.
+        // Output: warp e reads TMEM lane quadrant e, so thread (e, lane) holds head dimension
+        // 32 e + lane of every row and each row's 32 dimensions leave as one 64-byte store per
+        // warp.  Row metadata (output row index, 1 / l) is computed lane-parallel, 32 rows at a
+        // time, and broadcast with shuffles.  One thread waits on each mbarrier; the others
+        // learn the outcome at named barrier kBarEpilogue.
         const int eq = warp - kWarpEpi0;
+        const int et = tid - kWarpEpi0 * 32; // 0..127
+        const bool eleader = et == 0;
         const int dim = 32 * eq + lane;
         const uint32_t lane_base = static_cast<uint32_t>(32 * eq) << 16;
-        uint32_t nact = 0;
-        for (int64_t gi = g0; gi < L.n_groups; gi += gstep) {
-            const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
-            if (nU == 0)
-                continue;
-            const int h = L.gmeta[3 * gi + 1];
-            const int R = L.gsize[gi] * L.G;
-            const int npad = (R + 15) & ~15;
-            const uint32_t ob = nact & 1u;
+        // Q tile of group m: scaled, split into two E4M3 parts, written to buffer m % 2.
+        // Returns false when a wait gave up; nU_out < 0 marks the end.
+        auto prep_q = [&](uint32_t m, int &nU_out) -> bool {
+            const uint32_t jb = m % kNJ, qb = m & 1u;
+            if (!role_wait(&sm.job_full[jb], (m / kNJ) & 1u, &sm.abort_flag, eleader, kBarEpilogue,
+                           kEpiThreads))
+                return false;
+            GroupJob &J = sm.job[jb];
+            const int R = J.R;
+            nU_out = J.nU;
+            if (nU_out < 0)
+                return true;
+            // Q tile buffer qb was last read by the last S of group m - 2; the raw rows of
+            // group m have landed.
             bool got = true;
-            if (eq == 0 && lane == 0)
-                got = wait_bar(&sm.o_full[ob], (nact >> 1) & 1u, &sm.abort_flag) &&
-                      wait_bar(&sm.l_full[ob], (nact >> 1) & 1u, &sm.abort_flag);
+            if (eleader)
+                got = wait_bar(&sm.q_empty[qb], ((m >> 1) & 1u) ^ 1u, &sm.abort_flag) &&
+                      wait_bar(&sm.qraw_full, m & 1u, &sm.abort_flag);
+            if (bar_or(kBarEpilogue, kEpiThreads, !got))
+                return false;
+            // Row r of the tile is query head h G + r % G of query r / G.  Sixteen consecutive
+            // lanes hold one row (eight dims each) and agree on its scale.
+#pragma unroll
+            for (int rep = 0; rep < 1024 / kEpiThreads; ++rep) {
+                const int qn = et + kEpiThreads * rep;
+                const int row = qn >> 4, c = qn & 15;
+                const uint4 val = row < R ? *reinterpret_cast<const uint4 *>(sm.q_raw + row * 256 + c * 16)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+                uint32_t e = max_exp8(val);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1)
+                    e = max(e, __shfl_xor_sync(kFull, e, o));
+                const int sexp = q_scale_exp(e);
+                uint2 q1, q2;
+                split_q8(val, exp2i(sexp), q1, q2);
+                const uint32_t off = swz(row, c >> 1) + 8u * (c & 1);
+                *reinterpret_cast<uint2 *>(sm.q[qb][0] + off) = q1;
+                *reinterpret_cast<uint2 *>(sm.q[qb][1] + off) = q2;
+                if (c == 0)
+                    J.qexp[row] = sexp;
+            }
+            fence_proxy_async_smem();
+            warp_arrive(&sm.q_full[qb], lane);
+            warp_arrive(&sm.qraw_empty, lane);
+            return true;
+        };
+        uint32_t n = 0;
+        int nU = 0;
+        bool ok = prep_q(0, nU);
+        while (ok && nU >= 0) {
+            int nU_next = -1;
+            if (!prep_q(n + 1, nU_next))
+                break;
+            // output of group n
+            const uint32_t jb = n % kNJ, ob = n & 1u;
+            const GroupJob &J = sm.job[jb];
+            const int h = J.h, R = J.R;
+            const int npad = (R + 15) & ~15;
+            bool got = true;
+            if (eleader)
+                got = wait_bar(&sm.o_full[ob], (n >> 1) & 1u, &sm.abort_flag) &&
+                      wait_bar(&sm.l_full[ob], (n >> 1) & 1u, &sm.abort_flag);
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 break;
             tc_fence_after();
@@ -917,8 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int32_t orow = 0; // output row index tok * Hq + hq
                 if (r < R) {
                     const int mi = r / L.G;
-                    const int64_t tok = L.qids[gi * L.g + mi];
-                    orow = static_cast<int32_t>(tok * L.Hq + h * L.G + (r - mi * L.G));
+                    orow = J.tok[r] * L.Hq + h * L.G + (r - mi * L.G);
                     const float l_row = sm.lsum[ob][r][0] + sm.lsum[ob][r][1] + sm.lsum[ob][r][2] + sm.lsum[ob][r][3];
                     inv = l_row > 0.f ? L.v_scale / l_row : 0.f;
                 }
@@ -944,7 +1009,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             warp_arrive(&sm.o_free[ob], lane);
-            ++nact;
+            warp_arrive(&sm.job_empty[jb], lane);
+            ++n;
+            nU = nU_next;
         }
     }
 
