@@ -431,7 +431,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3 x e4m3 (S, Q split exactly in two e4m3 parts) and bf16 x bf16 (PV), fp32 accumulate",
+        "dtype": "e4m3 x e4m3 (S, Q split exactly in two e4m3 parts) and f16 x f16 (PV, P split in f16 hi + lo), fp32 accumulate",
         "data": "synthetic",
         "config": config_of(wl, args),
         "roofline": {
