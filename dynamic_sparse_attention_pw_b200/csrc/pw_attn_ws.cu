@@ -10,7 +10,7 @@
 // every element within 2^9 of the row's largest (an 8-bit bf16 significand is a 4-bit E4M3
 // significand plus a remainder of at most 4 bits); S = (q1 K^T + q2 K^T) 2^-s.  The product
 // O^T = V^T P^T runs on f16 operands: V decoded exactly (E4M3 is a subset of f16), P split
-// into f16 hi + lo parts.
+// into f16 hi + lo parts (the lo part stored negated, which the epilogue subtracts).
 //
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
 //   warps 0-3    decode   E4M3 V pages -> f16 operand tiles
@@ -26,9 +26,9 @@
 //                         the pages of step n - 1
 // Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
 // its scheduler delays its waits and issues.
-// O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and P_lo are stacked along N
-// (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, which the
-// epilogue adds.  A K stage is free once S is done, a V stage once it is decoded, an f16 V slot
+// O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and -P_lo are stacked along N
+// (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, and the
+// epilogue takes their difference.  A K stage is free once S is done, a V stage once it is decoded, an f16 V slot
 // once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
 // mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
 // other roles.
@@ -77,7 +77,7 @@ struct GroupJob {
 struct __align__(1024) WsSmem {
     uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
     uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] f16, swizzled
-    // [step parity][page of the step][P_hi rows 0..npad-1, P_lo rows npad..2npad-1][64 keys]
+    // [step parity][page of the step][P_hi rows 0..npad-1, -P_lo rows npad..2npad-1][64 keys]
     uint8_t p[2][2][128 * 128];
     // E4M3 K pages, 128-byte swizzled by the tensor copy; the two pages of a step sit in one
     // pair, so that they form one 128-row operand
@@ -282,7 +282,7 @@ __device__ __forceinline__ float quarter_max(const uint32_t (&sv)[16], int nq, b
 }
 
 // P of 16 keys of one row (the first nq allowed, the rest 0) into rows `row` (P_hi) and
-// npad + row (P_lo) of a page's P buffer; returns their sum.  Only rows < npad write.
+// npad + row (-P_lo) of a page's P buffer; returns their sum.  Only rows < npad write.
 __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float c, float negm,
                                         uint8_t *buf, int row, int qq, int npad)
 {
@@ -294,7 +294,7 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
             const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm));
             sum += p0 + p1;
-            split_pair_f16(p0, p1, hi[e], lo[e]);
+            split_pair_f16_neg(p0, p1, hi[e], lo[e]);
         }
     } else {
 #pragma unroll
@@ -302,7 +302,7 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm)) : 0.f;
             const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm)) : 0.f;
             sum += p0 + p1;
-            split_pair_f16(p0, p1, hi[e], lo[e]);
+            split_pair_f16_neg(p0, p1, hi[e], lo[e]);
         }
     }
     if (row < npad) {
@@ -1000,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float ie = __shfl_sync(kFull, inv, src);
                         const int32_t oe = __shfl_sync(kFull, orow, src);
                         if (c0 + e < R) {
-                            const float val = (__uint_as_float(ohi[e]) + __uint_as_float(olo[e])) * ie;
+                            const float val = (__uint_as_float(ohi[e]) - __uint_as_float(olo[e])) * ie;
                             L.O[static_cast<size_t>(oe) * kHeadDim + dim] =
                                 __bfloat16_as_ushort(__float2bfloat16_rn(val));
                         }
