@@ -71,7 +71,7 @@ struct GroupJob {
     int32_t pos[64];    // its position within its sequence
     int32_t qexp[64];   // its Q scale exponent (written by the decode warps)
     uint32_t word0[2][32]; // per query: its membership words of the first two union pages
-    int32_t b, h, R, nU, u0, pg0, pg1; // nU < 0: no further group
+    int32_t b, h, R, nU, u0, pg0, pg1, pg2, pg3; // union pages 0..3 (absent ones: pg0); nU < 0: no further group
 };
 
 struct __align__(1024) WsSmem {
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         struct GMeta {
             int64_t gi;
-            int b, h, gsz, R, u0, nU, pg0, pg1;
+            int b, h, gsz, R, u0, nU, pg0, pg1, pg2, pg3;
             int32_t tok_l, cu_b;   // lane l: query l of the group
             uint32_t w0_l, w1_l;   // lane l: its membership words of the first two union pages
         };
@@ -425,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m.cu_b = L.cu[b];
                 m.pg0 = L.union_pages[u0];
                 m.pg1 = nU > 1 ? L.union_pages[u0 + 1] : m.pg0;
+                m.pg2 = nU > 2 ? L.union_pages[u0 + 2] : m.pg0;
+                m.pg3 = nU > 3 ? L.union_pages[u0 + 3] : m.pg0;
                 const uint32_t *bitrow = L.bits + (static_cast<size_t>(m.tok_l) * L.Hkv + h) * L.words;
                 m.w0_l = lane < gsz ? __ldg(bitrow + (m.pg0 >> 5)) : 0u;
                 m.w1_l = lane < gsz ? __ldg(bitrow + (m.pg1 >> 5)) : 0u;
@@ -459,6 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     J.u0 = m->u0;
                     J.pg0 = m->pg0;
                     J.pg1 = m->pg1;
+                    J.pg2 = m->pg2;
+                    J.pg3 = m->pg3;
                 }
             }
             __syncwarp();
@@ -773,26 +777,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain factor
             const float inv = exp2i(-J.qexp[row]);
             const float crow_r = crow * inv, acrow_r = acrow * inv;
-            int pg_a = J.pg0, pg_b = J.pg1;
-            uint32_t word_a = valid ? J.word0[0][row / L.G] : 0u;
-            uint32_t word_b = valid ? J.word0[1][row / L.G] : 0u;
+            // Union page ids and my membership words, software-pipelined so that no step waits
+            // on a global load: at the top of each step the words of the next step's pages and
+            // the ids of the pages two steps ahead are requested; at its end, when they have
+            // landed, they move down one stage.
+            int pgA = J.pg0, pgB = J.pg1;     // this step
+            uint32_t wA = valid ? J.word0[0][row / L.G] : 0u;
+            uint32_t wB = valid ? J.word0[1][row / L.G] : 0u;
+            int pn0 = J.pg2, pn1 = J.pg3;     // next step (ids known)
+            uint32_t wn0 = 0u, wn1 = 0u;      // next step (words requested at the top of this one)
+            int pnn0 = pn0, pnn1 = pn1;       // two steps ahead (ids requested at the top of this one)
             warp_arrive(&sm.job_empty[jb], lane);
             const uint32_t ob = nact & 1u;
             const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
             float m_used = -INFINITY, l_part = 0.f;
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const int np = min(2, nU - s0);
-                const int pgA = pg_a, pgB = pg_b;
-                const uint32_t wA = word_a, wB = word_b;
-                // the next step's page ids and my membership words, fetched early
-                if (s0 + 2 < nU) {
-                    pg_a = L.union_pages[u0 + s0 + 2];
-                    word_a = valid ? __ldg(bitrow + (pg_a >> 5)) : 0u;
-                }
-                if (s0 + 3 < nU) {
-                    pg_b = L.union_pages[u0 + s0 + 3];
-                    word_b = valid ? __ldg(bitrow + (pg_b >> 5)) : 0u;
-                }
+                if (s0 + 2 < nU && valid)
+                    wn0 = __ldg(bitrow + (pn0 >> 5));
+                if (s0 + 3 < nU && valid)
+                    wn1 = __ldg(bitrow + (pn1 >> 5));
+                if (s0 + 4 < nU)
+                    pnn0 = L.union_pages[u0 + s0 + 4];
+                if (s0 + 5 < nU)
+                    pnn1 = L.union_pages[u0 + s0 + 5];
                 const uint32_t sb = stp & 1u;
                 const uint32_t it0 = it;
                 // every abort decision of this role is collective: a thread that left alone
@@ -844,7 +852,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (qq == 0)
                         sm.alpha[sb][row] = rescale ? alpha : 1.f;
-                    if (softmax_bar_or(rescale)) {
+                    // (at a group's first step no row has a max yet, so none rescales)
+                    if (s0 > 0 && softmax_bar_or(rescale)) {
                         // O^T[d, r] *= alpha[r] for both accumulator halves, once every product
                         // issued so far (those of the pages before this step) has completed.
                         ok = s0 == 0 || wait_pv(it0 - 1);
@@ -882,6 +891,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 warp_arrive(&sm.p_full[sb], lane);
                 it_prev0 = it0;
                 it += np;
+                pgA = pn0;
+                pgB = pn1;
+                wA = wn0;
+                wB = wn1;
+                pn0 = pnn0;
+                pn1 = pnn1;
             }
             if (!ok)
                 break;
