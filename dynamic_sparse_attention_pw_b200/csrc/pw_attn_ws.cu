@@ -947,8 +947,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 return false;
             // Row r of the tile is query head h G + r % G of query r / G.  Sixteen consecutive
-            // lanes hold one row (eight dims each) and agree on its scale.
-#pragma unroll
+            // lanes hold one row (eight dims each) and agree on its scale.  The loop stays rolled:
+            // this path has time to spare, and its unrolled code crowded the instruction cache
+            // that the softmax loop runs from.
+#pragma unroll 1
             for (int rep = 0; rep < 1024 / kEpiThreads; ++rep) {
                 const int qn = et + kEpiThreads * rep;
                 const int row = qn >> 4, c = qn & 15;
