@@ -133,6 +133,26 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
     }
 }
 
+// wait_bar for roles off the critical path (load, epilogue): between tries the thread sleeps,
+// so a long wait takes few issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool wait_bar_lazy(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    for (;;) {
+        __nanosleep(128);
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (*reinterpret_cast<volatile int32_t *>(abort_flag) != 0)
+            return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *reinterpret_cast<volatile int32_t *>(abort_flag) = 1;
+            return false;
+        }
+    }
+}
+
 // Named barriers, one per role that has more than one warp (0 is __syncthreads).
 constexpr uint32_t kBarSoftmax = 1, kBarDecode = 2, kBarEpilogue = 3;
 
@@ -803,13 +823,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pnn1 = L.union_pages[u0 + s0 + 5];
                 const uint32_t sb = stp & 1u;
                 const uint32_t it0 = it;
-                // every abort decision of this role is collective: a thread that left alone
-                // would strand the others at the named barrier or in a warp-wide TMEM load
-                ok = !sleader || wait_bar(&sm.s_done[sb], (stp >> 1) & 1u, &sm.abort_flag);
-                if (softmax_bar_or(!ok)) {
-                    ok = false;
-                    break;
-                }
+                // Every warp waits for S itself (all lanes poll, the warp decides by vote), so the
+                // warps are not lined up at a barrier here.  Every abort decision of this role is
+                // still collective (a thread that left alone would strand the others at the named
+                // barrier or in a warp-wide TMEM load): a warp whose wait gave up carries that to
+                // the vote below.
+                const bool s_ok = __all_sync(kFull, wait_bar(&sm.s_done[sb], (stp >> 1) & 1u, &sm.abort_flag));
                 if (pv_done < it_prev0)
                     pv_done = it_prev0;
                 // S of the step is read twice (for the max, then for P), one page at a time, so
@@ -834,7 +853,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool any = nqA > 0 || nqB > 0;
                 if (any)
                     lm *= acrow_r;
-                if (softmax_bar_or(any && lm > m_used + kRescaleLog2)) {
+                if (softmax_bar_or(!s_ok || (any && lm > m_used + kRescaleLog2))) {
+                    if (softmax_bar_or(!s_ok)) {
+                        ok = false;
+                        break;
+                    }
                     // slow path: the row's four threads agree on its max
                     sm.qmax[row][qq] = any ? lm : -INFINITY;
                     softmax_bar();
@@ -988,8 +1011,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int npad = (R + 15) & ~15;
             bool got = true;
             if (eleader)
-                got = wait_bar(&sm.o_full[ob], (n >> 1) & 1u, &sm.abort_flag) &&
-                      wait_bar(&sm.l_full[ob], (n >> 1) & 1u, &sm.abort_flag);
+                got = wait_bar_lazy(&sm.o_full[ob], (n >> 1) & 1u, &sm.abort_flag) &&
+                      wait_bar_lazy(&sm.l_full[ob], (n >> 1) & 1u, &sm.abort_flag);
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 break;
             tc_fence_after();
