@@ -339,6 +339,64 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
     return sum;
 }
 
+// The softmax role's slow path, taken when some row's scores exceed its running max by more
+// than 2^8 (always at a group's first step): the row's four threads agree on its max and, when
+// a row's max rises, O^T[d, r] *= alpha[r] for both accumulator halves once every product issued
+// so far (those of the pages up to wait_to) has completed.  Kept out of line so that the common
+// path of the softmax loop stays small in the instruction cache.  Every thread of the role calls
+// it; the state comes back by value.
+struct SlowOut {
+    float m_used, l_part;
+    uint32_t pv_done;
+    bool ok;
+};
+
+__device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, int hw, bool any, float lm,
+                                                  float m_used, float l_part, bool first_step, uint32_t sb,
+                                                  uint32_t wait_to, uint32_t pv_done, bool sleader,
+                                                  uint32_t o_addr, int npad)
+{
+    sm.qmax[row][qq] = any ? lm : -INFINITY;
+    softmax_bar();
+    const float M = fmaxf(fmaxf(sm.qmax[row][0], sm.qmax[row][1]), fmaxf(sm.qmax[row][2], sm.qmax[row][3]));
+    float alpha = 1.f;
+    bool rescale = false;
+    if (M > m_used + kRescaleLog2) {
+        if (m_used != -INFINITY) {
+            alpha = ex2(m_used - M);
+            rescale = true;
+            l_part *= alpha;
+        }
+        m_used = M;
+    }
+    if (qq == 0)
+        sm.alpha[sb][row] = rescale ? alpha : 1.f;
+    // (at a group's first step no row has a max yet, so none rescales)
+    if (!first_step && softmax_bar_or(rescale)) {
+        // v_empty[x % kNV] completes once per product of page x, and a parity wait is only
+        // unambiguous one phase ahead of what is known complete: step through the pages in order.
+        bool ok = true;
+        for (; pv_done <= wait_to && ok; ++pv_done)
+            if (sleader && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
+                ok = false;
+        if (softmax_bar_or(!ok))
+            return SlowOut{m_used, l_part, pv_done, false};
+        tc_fence_after();
+        for (int c0 = 16 * hw; c0 < 2 * npad; c0 += 32) {
+            uint32_t o[16];
+            tmem_ld16(o_addr + c0, o);
+            tmem_ld_wait16(o);
+            const int r0 = c0 < npad ? c0 : c0 - npad;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[sb][r0 + e]);
+            tmem_st16(o_addr + c0, o);
+        }
+        tmem_st_wait();
+    }
+    return SlowOut{m_used, l_part, pv_done, true};
+}
+
 // tmap_k: the K pages as a 2-D byte tensor [n_phys * Hkv * 64 rows][128], boxes of 64 x 128
 // with the 128-byte swizzle, so that one copy lands a page as the K-major operand of S.
 __global__ void __launch_bounds__(kThreads, 1)
@@ -751,19 +809,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float acrow = fabsf(crow);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
         uint32_t it = 0, stp = 0, nact = 0, it_prev0 = 0;
-        // Products known complete: pages [0, pv_done).  v_empty[x % kNV] completes once per
-        // product of page x, and a parity wait is only unambiguous one phase ahead of what is
-        // known complete, so wait_pv steps through the phases in page order.  Seeing S of step
-        // n also proves the products of step n - 2 complete (they were issued before it).  Only
-        // the leader waits (every thread advances pv_done alike); the collective vote that
-        // follows every call passes the outcome on.
+        // Products known complete: pages [0, pv_done).  Seeing S of step n proves the products
+        // of step n - 2 complete (they were issued before it); the slow path waits for the rest
+        // when it rescales.  Only the leader waits (every thread advances pv_done alike); the
+        // collective vote that follows passes the outcome on.
         uint32_t pv_done = 0;
-        auto wait_pv = [&](uint32_t x) -> bool { // product of page x complete
-            for (; pv_done <= x; ++pv_done)
-                if (sleader && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
-                    return false;
-            return true;
-        };
         auto allowed = [&](int pg, uint32_t word, int pos, int own) -> int { // keys of page pg in my quarter
             int n_allow = 0;
             if ((word >> (pg & 31)) & 1u)
@@ -858,44 +908,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    // slow path: the row's four threads agree on its max
-                    sm.qmax[row][qq] = any ? lm : -INFINITY;
-                    softmax_bar();
-                    const float M = fmaxf(fmaxf(sm.qmax[row][0], sm.qmax[row][1]),
-                                          fmaxf(sm.qmax[row][2], sm.qmax[row][3]));
-                    float alpha = 1.f;
-                    bool rescale = false;
-                    if (M > m_used + kRescaleLog2) {
-                        if (m_used != -INFINITY) {
-                            alpha = ex2(m_used - M);
-                            rescale = true;
-                            l_part *= alpha;
-                        }
-                        m_used = M;
-                    }
-                    if (qq == 0)
-                        sm.alpha[sb][row] = rescale ? alpha : 1.f;
-                    // (at a group's first step no row has a max yet, so none rescales)
-                    if (s0 > 0 && softmax_bar_or(rescale)) {
-                        // O^T[d, r] *= alpha[r] for both accumulator halves, once every product
-                        // issued so far (those of the pages before this step) has completed.
-                        ok = s0 == 0 || wait_pv(it0 - 1);
-                        if (softmax_bar_or(!ok)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        for (int c0 = 16 * hw; c0 < 2 * npad; c0 += 32) {
-                            uint32_t o[16];
-                            tmem_ld16(o_addr + c0, o);
-                            tmem_ld_wait16(o);
-                            const int r0 = c0 < npad ? c0 : c0 - npad;
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[sb][r0 + e]);
-                            tmem_st16(o_addr + c0, o);
-                        }
-                        tmem_st_wait();
+                    const SlowOut so = softmax_slow_path(sm, row, qq, hw, any, lm, m_used, l_part, s0 == 0, sb,
+                                                         it0 - 1, pv_done, sleader, o_addr, npad);
+                    m_used = so.m_used;
+                    l_part = so.l_part;
+                    pv_done = so.pv_done;
+                    if (!so.ok) {
+                        ok = false;
+                        break;
                     }
                 }
                 const float negm = m_used == -INFINITY ? 0.f : -m_used;
