@@ -133,9 +133,21 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int32_t
     }
 }
 
+// wait_bar for the waits outside the per-step loops of the softmax and MMA warps: the first try
+// inline, the spin out of line, so that these wait sites add little code.
+__device__ __noinline__ bool wait_bar_spin(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
+{
+    return wait_bar(bar, parity, abort_flag);
+}
+
+__device__ __forceinline__ bool wait_bar_c(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
+{
+    return mbar_try_wait(bar, parity) || wait_bar_spin(bar, parity, abort_flag);
+}
+
 // wait_bar for roles off the critical path (load, epilogue): between tries the thread sleeps,
 // so a long wait takes few issue slots from the warps that share its scheduler.
-__device__ __forceinline__ bool wait_bar_lazy(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
+__device__ __noinline__ bool wait_bar_lazy(uint64_t *bar, uint32_t parity, int32_t *abort_flag)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -189,7 +201,7 @@ __device__ __forceinline__ bool role_wait(uint64_t *bar, uint32_t parity, int32_
 {
     bool ok = true;
     if (leader)
-        ok = wait_bar(bar, parity, abort_flag);
+        ok = wait_bar_c(bar, parity, abort_flag);
     return !bar_or(id, n, !ok);
 }
 
@@ -468,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // membership words) stays off the other roles' path.  Every lane polls its mbarriers;
         // lane 0 issues the copies.
         auto lwait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return __all_sync(kFull, wait_bar(bar, parity, &sm.abort_flag));
+            return __all_sync(kFull, wait_bar_c(bar, parity, &sm.abort_flag));
         };
         struct GMeta {
             int64_t gi;
@@ -773,8 +785,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t st = it % kNSV, vs = it % kNV;
                 bool got = true;
                 if (tid == 0)
-                    got = wait_bar(&sm.vst_full[st], (it / kNSV) & 1u, &sm.abort_flag) &&
-                          wait_bar(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag);
+                    got = wait_bar_c(&sm.vst_full[st], (it / kNSV) & 1u, &sm.abort_flag) &&
+                          wait_bar_c(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag);
                 if (bar_or(kBarDecode, kDecThreads, !got)) {
                     ok = false;
                     break;
@@ -826,9 +838,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t jb = nact % kNJ;
             bool got = true;
             if (sleader) {
-                got = wait_bar(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag);
+                got = wait_bar_c(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag);
                 if (got && sm.job[jb].nU >= 0)
-                    got = wait_bar(&sm.q_full[nact & 1u], (nact >> 1) & 1u, &sm.abort_flag);
+                    got = wait_bar_c(&sm.q_full[nact & 1u], (nact >> 1) & 1u, &sm.abort_flag);
             }
             if (softmax_bar_or(!got)) {
                 ok = false;
@@ -945,7 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             // Publish the row-sum partials of this group for the epilogue warps.  lsum[ob] was
             // last read by the epilogue of group nact - 2, which released it with o_free[ob].
-            ok = !sleader || wait_bar(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
+            ok = !sleader || wait_bar_c(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
             if (softmax_bar_or(!ok)) {
                 ok = false;
                 break;
@@ -985,8 +997,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // group m have landed.
             bool got = true;
             if (eleader)
-                got = wait_bar(&sm.q_empty[qb], ((m >> 1) & 1u) ^ 1u, &sm.abort_flag) &&
-                      wait_bar(&sm.qraw_full, m & 1u, &sm.abort_flag);
+                got = wait_bar_c(&sm.q_empty[qb], ((m >> 1) & 1u) ^ 1u, &sm.abort_flag) &&
+                      wait_bar_c(&sm.qraw_full, m & 1u, &sm.abort_flag);
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 return false;
             // Row r of the tile is query head h G + r % G of query r / G.  Sixteen consecutive
