@@ -280,7 +280,10 @@ __global__ void __launch_bounds__(128) k_greedy(
 }
 
 // ---------------------------------------------------------------------------------------
-// k_union_offsets: single block; exclusive scan of ucount -> union_off[0..n].
+// k_union_offsets: single block; exclusive scan of ucount -> union_off[0..n].  Thread t owns
+// the contiguous range [t c, (t + 1) c), c a multiple of 4, read and written as int4 where both
+// arrays are 16-byte aligned: one pass for the range sums, a block scan of the sums, one pass
+// for the offsets.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_union_offsets(const int32_t *__restrict__ ucount,
                                                         int64_t n, int64_t cap,
@@ -289,11 +292,17 @@ __global__ void __launch_bounds__(1024) k_union_offsets(const int32_t *__restric
 {
     __shared__ long long wsum[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t chunk = (n + blockDim.x - 1) / blockDim.x;
-    const int64_t s = static_cast<int64_t>(tid) * chunk;
+    const int64_t chunk = ((n + blockDim.x - 1) / blockDim.x + 3) & ~static_cast<int64_t>(3);
+    const int64_t s = min(n, static_cast<int64_t>(tid) * chunk);
     const int64_t e = min(n, s + chunk);
+    const bool vec = ((reinterpret_cast<uintptr_t>(ucount) | reinterpret_cast<uintptr_t>(union_off)) & 15) == 0;
+    const int64_t ev = vec ? s + ((e - s) & ~static_cast<int64_t>(3)) : s; // end of the int4 part
     long long local = 0;
-    for (int64_t i = s; i < e; ++i)
+    for (int64_t i = s; i < ev; i += 4) {
+        const int4 v = *reinterpret_cast<const int4 *>(ucount + i);
+        local += static_cast<long long>(v.x) + v.y + v.z + v.w;
+    }
+    for (int64_t i = ev; i < e; ++i)
         local += ucount[i];
     long long incl = local;
 #pragma unroll
@@ -319,7 +328,17 @@ __global__ void __launch_bounds__(1024) k_union_offsets(const int32_t *__restric
     }
     __syncthreads();
     long long base = (warp > 0 ? wsum[warp - 1] : 0) + incl - local;
-    for (int64_t i = s; i < e; ++i) {
+    for (int64_t i = s; i < ev; i += 4) {
+        const int4 v = *reinterpret_cast<const int4 *>(ucount + i);
+        int4 o;
+        o.x = static_cast<int32_t>(base);
+        o.y = static_cast<int32_t>(base + v.x);
+        o.z = static_cast<int32_t>(base + v.x + v.y);
+        o.w = static_cast<int32_t>(base + v.x + v.y + v.z);
+        base += static_cast<long long>(v.x) + v.y + v.z + v.w;
+        *reinterpret_cast<int4 *>(union_off + i) = o;
+    }
+    for (int64_t i = ev; i < e; ++i) {
         union_off[i] = static_cast<int32_t>(base);
         base += ucount[i];
     }
