@@ -573,25 +573,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                          L.Q + (static_cast<size_t>(m.tok_l) * L.Hq + m.h * L.G) * kHeadDim,
                          static_cast<uint32_t>(L.G) * 256u, &sm.qraw_full);
         };
-        uint32_t it = 0, stp = 0, nj = 0;
-        bool stop = false;
+        uint32_t it = 0, stp = 0;
+        bool stop = false, has_cur = false;
         GMeta cur{}, nxt{};
-        bool has_cur = next_group(g0, cur);
-        if (has_cur)
-            stop = !publish(0, &cur) || !lwait(&sm.qraw_empty, 1u);
-        else
-            stop = !publish(0, nullptr);
-        if (has_cur && !stop)
-            copy_q(0, cur);
-        while (has_cur && !stop) {
-            const bool has_nxt = next_group(cur.gi + gstep, nxt);
-            if (!publish(nj + 1, has_nxt ? &nxt : nullptr)) {
+        int64_t gi_next = g0;
+        // Iteration n publishes job n (the next group's record, or the end marker), then issues
+        // the pages of job n - 1 and, as soon as the raw Q buffer is free, job n's Q rows.  One
+        // call site for each keeps this role's code small.
+        for (uint32_t n = 0; !stop; ++n) {
+            const bool has_nxt = next_group(gi_next, nxt);
+            if (!publish(n, has_nxt ? &nxt : nullptr)) {
                 stop = true;
                 break;
             }
-            bool q_pending = has_nxt; // Q rows of job nj + 1, once job nj's raw rows are used
-            const uint32_t q_parity = (nj & 1u); // phase nj of qraw_empty (released by job nj's split)
-            const int b = cur.b, h = cur.h, u0 = cur.u0, nU = cur.nU;
+            bool q_pending = has_nxt; // Q rows of job n, once job n - 1's raw rows are used
+            // phase n - 1 of qraw_empty (released by job n - 1's split; for n = 0 the phase
+            // before the first, which reads as complete)
+            const uint32_t q_parity = (n & 1u) ^ 1u;
+            const int b = cur.b, h = cur.h, u0 = cur.u0, nU = has_cur ? cur.nU : 0;
             for (int j0 = 0; j0 < nU && !stop; j0 += 32) {
                 int phys = 0;
                 if (j0 + lane < nU) {
@@ -637,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     // the next job's Q rows, as soon as the raw buffer is free (no wait here)
                     if (!stop && q_pending && __all_sync(kFull, mbar_try_wait(&sm.qraw_empty, q_parity))) {
-                        copy_q(nj + 1, nxt);
+                        copy_q(n, nxt);
                         q_pending = false;
                     }
                 }
@@ -647,11 +646,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     stop = true;
                     break;
                 }
-                copy_q(nj + 1, nxt);
+                copy_q(n, nxt);
             }
+            if (!has_nxt)
+                break;
             cur = nxt;
-            has_cur = has_nxt;
-            ++nj;
+            has_cur = true;
+            gi_next = nxt.gi + gstep;
         }
     } else if (warp == kWarpMma) {
         // ---------------- MMA issue: the warp runs in lockstep, one elected lane issues ----------------
@@ -1029,14 +1030,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             warp_arrive(&sm.qraw_empty, lane);
             return true;
         };
-        uint32_t n = 0;
-        int nU = 0;
-        bool ok = prep_q(0, nU);
-        while (ok && nU >= 0) {
-            int nU_next = -1;
-            if (!prep_q(n + 1, nU_next))
+        // Iteration m prepares the Q tile of job m, then outputs group m - 1; one call site for
+        // each keeps this role's code small.
+        bool prev = false; // group m - 1 exists
+        for (uint32_t m = 0;; ++m) {
+            int nU_m = -1;
+            if (!prep_q(m, nU_m))
                 break;
-            // output of group n
+            if (!prev) {
+                if (nU_m < 0)
+                    break;
+                prev = true;
+                continue;
+            }
+            // output of group n = m - 1
+            const uint32_t n = m - 1;
             const uint32_t jb = n % kNJ, ob = n & 1u;
             const GroupJob &J = sm.job[jb];
             const int h = J.h, R = J.R;
@@ -1082,8 +1090,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             warp_arrive(&sm.o_free[ob], lane);
             warp_arrive(&sm.job_empty[jb], lane);
-            ++n;
-            nU = nU_next;
+            if (nU_m < 0)
+                break;
         }
     }
 
