@@ -15,21 +15,25 @@
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
 //   warps 0-3    decode   E4M3 V pages -> f16 operand tiles
 //   warps 4-11   softmax  S -> P for each step of one or two pages (four threads per row,
-//                         16 keys of each page each), lazy O^T rescale, per-row sums of each group
+//                         16 keys of each page each), lazy O^T rescale (out of line), per-row
+//                         sums of each group
 //   warps 12-15  epilogue Q tile of the next group (scaled, split into two E4M3 parts) while
 //                         the current one runs, then O^T of the finished group -> bf16 rows of O
 //                         (one warp per TMEM lane quadrant)
 //   warp 16      load     one group ahead: group records (rows, positions, first membership
-//                         words), the next group's Q rows by TMA, and the union pages: K through
-//                         a tensor map with the 128-byte swizzle the MMA reads, V by bulk copy
+//                         words, first page ids), the next group's Q rows by TMA, and the union
+//                         pages: K through a tensor map with the 128-byte swizzle the MMA reads,
+//                         V by bulk copy
 //   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O^T += V^T P^T for
 //                         the pages of step n - 1
 // Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
-// its scheduler delays its waits and issues.
+// its scheduler delays its waits and issues.  Compact code on purpose too: five roles run
+// different code on each scheduler, so cold paths stay out of line or rolled and each role's
+// loop calls its steps from one place, leaving the instruction cache to the hot loops.
 // O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and -P_lo are stacked along N
 // (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, and the
-// epilogue takes their difference.  A K stage is free once S is done, a V stage once it is decoded, an f16 V slot
-// once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
+// epilogue takes their difference.  A K stage is free once S is done, a V stage once it is
+// decoded, an f16 V slot once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
 // mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
 // other roles.
 #include <cstdint>
@@ -69,7 +73,7 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 struct GroupJob {
     int32_t tok[64];    // query token of each tile row (rows >= R: 0)
     int32_t pos[64];    // its position within its sequence
-    int32_t qexp[64];   // its Q scale exponent (written by the decode warps)
+    int32_t qexp[64];   // its Q scale exponent (written by the epilogue warps with the Q tile)
     uint32_t word0[2][32]; // per query: its membership words of the first two union pages
     int32_t b, h, R, nU, u0, pg0, pg1, pg2, pg3; // union pages 0..3 (absent ones: pg0); nU < 0: no further group
 };
