@@ -108,23 +108,6 @@ __device__ __forceinline__ void decode_page_f16(const uint8_t *src, uint8_t (*ds
     }
 }
 
-// p -> (hi, -lo) f16 halves of two packed words: hi = p rounded to f16, and nlo = hi - p (exact
-// in f32) rounded to f16, which is -lo exactly since rounding to nearest is symmetric.  The
-// difference takes one mixed-precision subtract per value (the f16 operand is widened exactly),
-// so the split costs four instructions per pair.  For p in [2^-3, 256] the pair carries about 22
-// significant bits; below, the absolute error stays under 2^-25.
-__device__ __forceinline__ void split_pair_f16_neg(float p0, float p1, uint32_t &hi2, uint32_t &nlo2)
-{
-    asm("{\n\t.reg .b16 h0, h1;\n\t.reg .f32 d0, d1;\n\t"
-        "cvt.rn.f16x2.f32 %0, %3, %2;\n\t"
-        "mov.b32 {h0, h1}, %0;\n\t"
-        "sub.f32.f16 d0, h0, %2;\n\t"
-        "sub.f32.f16 d1, h1, %3;\n\t"
-        "cvt.rn.f16x2.f32 %1, d1, d0;\n\t}"
-        : "=r"(hi2), "=r"(nlo2)
-        : "f"(p0), "f"(p1));
-}
-
 __device__ __forceinline__ float ex2(float x)
 {
     float y;

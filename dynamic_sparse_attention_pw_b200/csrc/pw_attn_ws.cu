@@ -9,33 +9,34 @@
 // is scaled by a power of two and split into two E4M3 parts, q' = q1 + q2, which is exact for
 // every element within 2^9 of the row's largest (an 8-bit bf16 significand is a 4-bit E4M3
 // significand plus a remainder of at most 4 bits); S = (q1 K^T + q2 K^T) 2^-s.  The product
-// O^T = V^T P^T runs on f16 operands: V decoded exactly (E4M3 is a subset of f16), P split
-// into f16 hi + lo parts (the lo part stored negated, which the epilogue subtracts).
+// O += P V runs on f16 operands with P read from TMEM: P split into f16 hi + lo parts, both
+// multiplied into the one accumulator, and V decoded exactly (E4M3 is a subset of f16).
 //
 // One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
 //   warps 0-3    decode   E4M3 V pages -> f16 operand tiles
 //   warps 4-11   softmax  S -> P for each step of one or two pages (four threads per row,
-//                         16 keys of each page each), lazy O^T rescale (out of line), per-row
-//                         sums of each group
+//                         16 keys of each page each), written back to TMEM over the S it came
+//                         from; lazy O rescale (out of line); per-row sums of each group
 //   warps 12-15  epilogue Q tile of the next group (scaled, split into two E4M3 parts) while
-//                         the current one runs, then O^T of the finished group -> bf16 rows of O
+//                         the current one runs, then O of the finished group -> bf16 rows of O
 //                         (one warp per TMEM lane quadrant)
 //   warp 16      load     one group ahead: group records (rows, positions, first membership
 //                         words, first page ids), the next group's Q rows by TMA, and the union
 //                         pages: K through a tensor map with the 128-byte swizzle the MMA reads,
 //                         V by bulk copy
-//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O^T += V^T P^T for
-//                         the pages of step n - 1
+//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O += P V for the
+//                         pages of step n - 1
 // Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
 // its scheduler delays its waits and issues.  Compact code on purpose too: five roles run
 // different code on each scheduler, so cold paths stay out of line or rolled and each role's
 // loop calls its steps from one place, leaving the instruction cache to the hot loops.
-// O^T = V^T P^T puts the head dimension on the 128 MMA rows; P_hi and -P_lo are stacked along N
-// (N = 2 * rows), so one product per k-step reads V once and accumulates both halves, and the
-// epilogue takes their difference.  A K stage is free once S is done, a V stage once it is
-// decoded, an f16 V slot once the product is done.  O^T is double-buffered across groups.  Every hand-off is an
-// mbarrier; every wait is bounded and, when it runs out, sets an abort flag that releases the
-// other roles.
+// TMEM holds two S buffers and two O buffers (M = 64 layout: row r at lane 32 (r / 16) + r % 16).
+// The P of a step replaces its S in place, as the A operand of the products (keys 2j and 2j + 1
+// of a 16-key block packed in column j: P_hi in a block's first 8 columns, P_lo in the next 8);
+// S two steps later overwrites it only after those products are done.  A K stage is free once S
+// is done, a V stage once it is decoded, an f16 V slot once the product is done.  O is
+// double-buffered across groups.  Every hand-off is an mbarrier; every wait is bounded and, when
+// it runs out, sets an abort flag that releases the other roles.
 #include <cstdint>
 #include <cuda.h> // CUtensorMap and its enums (the encoder itself is fetched at run time)
 #include <cuda_bf16.h>
@@ -63,7 +64,7 @@ constexpr int kWarpSm0 = kDecThreads / 32, kWarpEpi0 = kWarpSm0 + 8, kWarpLoad =
 constexpr int kThreads = 32 * (kWarpMma + 1);
 static_assert(kWarpSm0 % 4 == 0, "softmax warp w must sit in TMEM lane quadrant w % 4");
 static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
-constexpr uint32_t kTmemCols = 512; // S[0..1] at columns 0 / 128, O^T[0..1] at 256 / 384
+constexpr uint32_t kTmemCols = 512; // S / P [0..1] at columns 0 / 128, O[0..1] at 256 / 384
 constexpr uint32_t kColS = 128;     // one S step: two pages of 64 keys
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
@@ -81,15 +82,12 @@ struct GroupJob {
 struct __align__(1024) WsSmem {
     uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
     uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] f16, swizzled
-    // [step parity][page of the step][P_hi rows 0..npad-1, -P_lo rows npad..2npad-1][64 keys]
-    uint8_t p[2][2][128 * 128];
     // E4M3 K pages, 128-byte swizzled by the tensor copy; the two pages of a step sit in one
     // pair, so that they form one 128-row operand
     uint8_t stage_k[kNKP][2][kPageBytes];
     uint8_t stage_v[kNSV][kPageBytes]; // E4M3 V pages, row-major
     uint8_t q_raw[64 * 256];           // bf16 Q rows of the next group, row r at 256 r
     GroupJob job[kNJ];
-    float alpha[2][64];
     float qmax[64][4];    // per-row partial maxima exchanged by the row's four threads
     float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
     uint64_t job_full[kNJ], job_empty[kNJ];
@@ -98,6 +96,7 @@ struct __align__(1024) WsSmem {
     uint64_t vst_full[kNSV], vst_empty[kNSV];
     uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
     uint64_t s_done[2];                 // s_done[n % 2]: S of step n complete
+    uint64_t pvs_done[2];               // pvs_done[n % 2]: the products of step n complete
     uint64_t p_full[2];                 // p_full[n % 2]: P of both pages of step n written
     uint64_t q_full[2], q_empty[2];
     uint64_t o_full[2]; // last product of the group in O buffer b complete
@@ -317,10 +316,79 @@ __device__ __forceinline__ float quarter_max(const uint32_t (&sv)[16], int nq, b
     return lm;
 }
 
-// P of 16 keys of one row (the first nq allowed, the rest 0) into rows `row` (P_hi) and
-// npad + row (-P_lo) of a page's P buffer; returns their sum.  Only rows < npad write.
+// p -> (hi, lo) f16 halves of two packed words: hi = p rounded to f16, lo = p - hi (exact in
+// f32, formed by one mixed-precision multiply-add with the f16 operand widened exactly) rounded
+// to f16.  For p in [2^-3, 256] the pair carries about 22 significant bits; below, the absolute
+// error stays under 2^-25.
+__device__ __forceinline__ void split_pair_f16_pos(float p0, float p1, uint32_t &hi2, uint32_t &lo2)
+{
+    asm("{\n\t.reg .b16 h0, h1, m1;\n\t.reg .f32 d0, d1;\n\t"
+        "mov.b16 m1, 0xBC00;\n\t" // -1.0 in f16
+        "cvt.rn.f16x2.f32 %0, %3, %2;\n\t"
+        "mov.b32 {h0, h1}, %0;\n\t"
+        "fma.rn.f32.f16 d0, h0, m1, %2;\n\t"
+        "fma.rn.f32.f16 d1, h1, m1, %3;\n\t"
+        "cvt.rn.f16x2.f32 %1, d1, d0;\n\t}"
+        : "=r"(hi2), "=r"(lo2)
+        : "f"(p0), "f"(p1));
+}
+
+// 16 lanes x 32 bit, two column halves (the 16x32bx2 shape with a split of 16 columns): lanes
+// 0-15 of the warp write 8 columns from the address's column, lanes 16-31 from 16 columns on.
+__device__ __forceinline__ void tmem_st_16x32bx2_x8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], 16, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+// The same shape, 32 columns per half (split of 32 columns).
+__device__ __forceinline__ void tmem_ld_16x32bx2_x32s(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+                   "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+                   "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st_16x32bx2_x32s(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+                 "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+                 "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),
+                 "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+                 : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem] with kind::f16: A is read from TMEM (for M = 64, row r at lane
+// 32 (r / 16) + r % 16, keys 2j and 2j + 1 packed in column j), B from a shared-memory
+// descriptor.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// P of the 16 keys of one row that this thread read from TMEM at s_addr (the first nq allowed,
+// the rest 0), written back over those columns as the A operand of O += P V: P_hi in the first
+// 8 columns, P_lo in the last 8 (for lanes 16-31 of the warp, 16 columns further on, as they were
+// read).  Returns the keys' sum.
 __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float c, float negm,
-                                        uint8_t *buf, int row, int qq, int npad)
+                                        uint32_t s_addr)
 {
     uint32_t hi[8], lo[8];
     float sum = 0.f;
@@ -330,7 +398,7 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
             const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm));
             sum += p0 + p1;
-            split_pair_f16_neg(p0, p1, hi[e], lo[e]);
+            split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
     } else {
 #pragma unroll
@@ -338,27 +406,18 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm)) : 0.f;
             const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm)) : 0.f;
             sum += p0 + p1;
-            split_pair_f16_neg(p0, p1, hi[e], lo[e]);
+            split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
     }
-    if (row < npad) {
-        uint8_t *phi = buf, *plo = buf + npad * 128;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const uint32_t o = swz(row, 2 * qq + cc);
-            *reinterpret_cast<uint4 *>(phi + o) =
-                make_uint4(hi[4 * cc], hi[4 * cc + 1], hi[4 * cc + 2], hi[4 * cc + 3]);
-            *reinterpret_cast<uint4 *>(plo + o) =
-                make_uint4(lo[4 * cc], lo[4 * cc + 1], lo[4 * cc + 2], lo[4 * cc + 3]);
-        }
-    }
+    tmem_st_16x32bx2_x8(s_addr, hi);
+    tmem_st_16x32bx2_x8(s_addr + 8, lo);
     return sum;
 }
 
 // The softmax role's slow path, taken when some row's scores exceed its running max by more
 // than 2^8 (always at a group's first step): the row's four threads agree on its max and, when
-// a row's max rises, O^T[d, r] *= alpha[r] for both accumulator halves once every product issued
-// so far (those of the pages up to wait_to) has completed.  Kept out of line so that the common
+// a row's max rises, O[r, :] *= alpha[r] once every product issued so far (those of the pages up
+// to wait_to) has completed.  Kept out of line so that the common
 // path of the softmax loop stays small in the instruction cache.  Every thread of the role calls
 // it; the state comes back by value.
 struct SlowOut {
@@ -368,9 +427,9 @@ struct SlowOut {
 };
 
 __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, int hw, bool any, float lm,
-                                                  float m_used, float l_part, bool first_step, uint32_t sb,
+                                                  float m_used, float l_part, bool first_step,
                                                   uint32_t wait_to, uint32_t pv_done, bool sleader,
-                                                  uint32_t o_addr, int npad)
+                                                  uint32_t o_addr)
 {
     sm.qmax[row][qq] = any ? lm : -INFINITY;
     softmax_bar();
@@ -385,8 +444,6 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
         }
         m_used = M;
     }
-    if (qq == 0)
-        sm.alpha[sb][row] = rescale ? alpha : 1.f;
     // (at a group's first step no row has a max yet, so none rescales)
     if (!first_step && softmax_bar_or(rescale)) {
         // v_empty[x % kNV] completes once per product of page x, and a parity wait is only
@@ -397,17 +454,16 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
                 ok = false;
         if (softmax_bar_or(!ok))
             return SlowOut{m_used, l_part, pv_done, false};
+        // O[r, :] *= alpha[r]: the row sits in this warp's lanes, and its four threads take 32
+        // head dimensions each (lanes 0-15 dims 64 hw .. 64 hw + 31, lanes 16-31 the next 32).
         tc_fence_after();
-        for (int c0 = 16 * hw; c0 < 2 * npad; c0 += 32) {
-            uint32_t o[16];
-            tmem_ld16(o_addr + c0, o);
-            tmem_ld_wait16(o);
-            const int r0 = c0 < npad ? c0 : c0 - npad;
+        uint32_t o[32];
+        tmem_ld_16x32bx2_x32s(o_addr + 64 * hw, o);
+        tmem_ld_wait(o);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                o[e] = __float_as_uint(__uint_as_float(o[e]) * sm.alpha[sb][r0 + e]);
-            tmem_st16(o_addr + c0, o);
-        }
+        for (int e = 0; e < 32; ++e)
+            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st_16x32bx2_x32s(o_addr + 64 * hw, o);
         tmem_st_wait();
     }
     return SlowOut{m_used, l_part, pv_done, true};
@@ -451,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_done[s], 1);
+            mbar_init(&sm.pvs_done[s], 1);
             mbar_init(&sm.p_full[s], kSmThreads / 32);
             mbar_init(&sm.q_full[s], kEpiThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
@@ -669,18 +726,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             return __all_sync(kFull, ok);
         };
         const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
-        const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // MN-major V^T
+        const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // V, MN-major (dims contiguous)
         uint32_t it = 0, stp = 0, nact = 0;
         bool have_prev = false, ok = true;
         // the step whose products are still to issue, kept in scalars
-        uint32_t pv_it0 = 0, pv_stp = 0, pv_np = 0, pv_nact = 0, pv_npad = 16;
+        uint32_t pv_it0 = 0, pv_stp = 0, pv_np = 0, pv_nact = 0;
         bool pv_first = false, pv_last = false;
         auto issue_pv = [&]() -> bool {
             const uint32_t ob = pv_nact & 1u;
             if (!wwait(&sm.p_full[pv_stp & 1u], (pv_stp >> 1) & 1u))
                 return false;
-            const uint32_t idesc = idesc_f16_f32(128, static_cast<int>(2 * pv_npad), true, false);
+            // O (M = 64 rows, N = 128 dims) += P_hi V + P_lo V, P read from TMEM where the
+            // softmax wrote it (the step's S buffer), V (K = keys, N = dims) from its MN-major
+            // f16 tile.
+            constexpr uint32_t idesc = idesc_f16_f32(64, 128, false, true);
             const uint32_t d = tmem + kColO + 128 * ob;
+            const uint32_t pa = tmem + kColS * (pv_stp & 1u);
             for (uint32_t k = 0; k < pv_np; ++k) {
                 const uint32_t page = pv_it0 + k, vs = page % kNV;
                 const bool first = pv_first && k == 0;
@@ -688,15 +749,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (first && !wwait(&sm.o_free[ob], ((pv_nact >> 1) & 1u) ^ 1u)))
                     return false;
                 tc_fence_after();
-                const uint64_t ad = desc_add(dmn, smem_u32(&sm.v[vs][0][0]));
-                const uint64_t bd = desc_add(dsw, smem_u32(sm.p[pv_stp & 1u][k]));
+                const uint64_t bd = desc_add(dmn, smem_u32(&sm.v[vs][0][0]));
                 if (elect_one()) {
+                    // keys 16 kk .. 16 kk + 15: P_hi in columns 16 kk .. 16 kk + 7 of the page,
+                    // P_lo in the next 8
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_ss(d, ad + 128u * kk, bd + 2u * kk, idesc, (first && kk == 0) ? 0u : 1u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t a = pa + 64 * k + 16 * kk;
+                        mma_f16_ts(d, a, bd + 128u * kk, idesc, (first && kk == 0) ? 0u : 1u);
+                        mma_f16_ts(d, a + 8, bd + 128u * kk, idesc, 1u);
+                    }
                     mma_commit(&sm.v_empty[vs]);
-                    if (pv_last && k + 1 == pv_np)
-                        mma_commit(&sm.o_full[ob]);
+                    if (k + 1 == pv_np) {
+                        mma_commit(&sm.pvs_done[pv_stp & 1u]);
+                        if (pv_last)
+                            mma_commit(&sm.o_full[ob]);
+                    }
                 }
                 __syncwarp();
             }
@@ -708,13 +776,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            const int R = sm.job[jb].R, nU = sm.job[jb].nU;
+            const int nU = sm.job[jb].nU;
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sm.job_empty[jb]);
             if (nU < 0)
                 break;
-            const uint32_t npad = static_cast<uint32_t>((R + 15) & ~15);
             const uint32_t qb = nact & 1u;
             if (!wwait(&sm.q_full[qb], (nact >> 1) & 1u)) {
                 ok = false;
@@ -725,9 +792,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const uint32_t np = static_cast<uint32_t>(min(2, nU - s0));
                 const uint32_t kp = stp % kNKP, sb = stp & 1u;
-                // S buffer sb was last read by the softmax of step stp - 2, before it wrote the
-                // P that the products issued in the previous iteration waited for.
-                if (!wwait(&sm.kst_full[kp], (stp / kNKP) & 1u)) {
+                // S buffer sb holds the P of step stp - 2 (written by the softmax after it read S
+                // there): S may overwrite it once the products of that step have read it.  Their
+                // phase is one ahead of the one waited for two steps ago.
+                if (!wwait(&sm.kst_full[kp], (stp / kNKP) & 1u) ||
+                    (stp >= 2 && !wwait(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u))) {
                     ok = false;
                     break;
                 }
@@ -757,7 +826,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pv_stp = stp;
                 pv_np = np;
                 pv_nact = nact;
-                pv_npad = npad;
                 pv_first = s0 == 0;
                 pv_last = s0 + static_cast<int>(np) == nU;
                 have_prev = true;
@@ -856,7 +924,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nU < 0)
                 break;
             const int h = J.h, R = J.R, u0 = J.u0;
-            const int npad = (R + 15) & ~15;
             const bool valid = row < R;
             const int32_t tok = J.tok[row];
             const int pos = J.pos[row], own = pos >> 6;
@@ -925,8 +992,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    const SlowOut so = softmax_slow_path(sm, row, qq, hw, any, lm, m_used, l_part, s0 == 0, sb,
-                                                         it0 - 1, pv_done, sleader, o_addr, npad);
+                    const SlowOut so = softmax_slow_path(sm, row, qq, hw, any, lm, m_used, l_part, s0 == 0,
+                                                         it0 - 1, pv_done, sleader, o_addr);
                     m_used = so.m_used;
                     l_part = so.l_part;
                     pv_done = so.pv_done;
@@ -936,17 +1003,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 const float negm = m_used == -INFINITY ? 0.f : -m_used;
-                // P buffers [sb][*] were last read by the products of step stp - 2, complete
-                // since S of this step (issued after them) is.
+                // P of each page goes back over that page's S columns (each thread over the 16 it
+                // read), where the products read it as their A operand.  The products of step
+                // stp - 2 read the same columns as P before S of this step overwrote them (the
+                // tensor pipe keeps issue order).
                 for (int k = 0; k < np; ++k) {
                     uint32_t sv[16];
                     tc_fence_after();
                     tmem_ld_16x32bx2_x16(s_addr + 64 * k, sv);
                     tmem_ld_wait16(sv);
-                    l_part += emit_p(sv, k == 0 ? nqA : nqB, crow_r, negm, sm.p[sb][k], row, qq, npad);
+                    l_part += emit_p(sv, k == 0 ? nqA : nqB, crow_r, negm, s_addr + 64 * k);
                 }
-                tc_fence_before();
-                fence_proxy_async_smem();
+                tmem_st_wait();
                 tc_fence_before();
                 warp_arrive(&sm.p_full[sb], lane);
                 it_prev0 = it0;
@@ -984,7 +1052,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int eq = warp - kWarpEpi0;
         const int et = tid - kWarpEpi0 * 32; // 0..127
         const bool eleader = et == 0;
-        const int dim = 32 * eq + lane;
         const uint32_t lane_base = static_cast<uint32_t>(32 * eq) << 16;
         // Q tile of group m: scaled, split into two E4M3 parts, written to buffer m % 2.
         // Returns false when a wait gave up; nU_out < 0 marks the end.
@@ -1052,43 +1119,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t jb = n % kNJ, ob = n & 1u;
             const GroupJob &J = sm.job[jb];
             const int h = J.h, R = J.R;
-            const int npad = (R + 15) & ~15;
             bool got = true;
             if (eleader)
                 got = wait_bar_lazy(&sm.o_full[ob], (n >> 1) & 1u, &sm.abort_flag) &&
                       wait_bar_lazy(&sm.l_full[ob], (n >> 1) & 1u, &sm.abort_flag);
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 break;
+            // O in TMEM: row r at lane 32 (r / 16) + r % 16 of quadrant r / 16, head dimensions
+            // along the columns.  Warp eq takes rows 16 eq .. 16 eq + 15; lanes 0-15 and 16-31
+            // take 32 dimensions each per load, so each thread writes 64 contiguous bytes of a row.
             tc_fence_after();
             const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
-            for (int cb = 0; cb < npad; cb += 32) {
-                const int r = cb + lane;
-                float inv = 0.f;
-                int32_t orow = 0; // output row index tok * Hq + hq
+            const int r = 16 * eq + (lane & 15), half = lane >> 4;
+            float inv = 0.f;
+            uint16_t *orow = nullptr;
+            if (r < R) {
+                const int mi = r / L.G;
+                orow = L.O + static_cast<size_t>(J.tok[r] * L.Hq + h * L.G + (r - mi * L.G)) * kHeadDim;
+                const float l_row = sm.lsum[ob][r][0] + sm.lsum[ob][r][1] + sm.lsum[ob][r][2] + sm.lsum[ob][r][3];
+                inv = l_row > 0.f ? L.v_scale / l_row : 0.f;
+            }
+#pragma unroll 1
+            for (int cb = 0; cb < kHeadDim; cb += 64) {
+                uint32_t o[32];
+                tmem_ld_16x32bx2_x32s(o_addr + cb, o);
+                tmem_ld_wait(o);
                 if (r < R) {
-                    const int mi = r / L.G;
-                    orow = J.tok[r] * L.Hq + h * L.G + (r - mi * L.G);
-                    const float l_row = sm.lsum[ob][r][0] + sm.lsum[ob][r][1] + sm.lsum[ob][r][2] + sm.lsum[ob][r][3];
-                    inv = l_row > 0.f ? L.v_scale / l_row : 0.f;
-                }
-                const int cend = min(cb + 32, npad);
-                for (int c0 = cb; c0 < cend; c0 += 16) {
-                    uint32_t ohi[16], olo[16];
-                    tmem_ld16(o_addr + c0, ohi);
-                    tmem_ld16(o_addr + npad + c0, olo);
-                    tmem_ld_wait16(ohi);
-                    tmem_ld_wait16(olo);
+                    uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int src = c0 - cb + e;
-                        const float ie = __shfl_sync(kFull, inv, src);
-                        const int32_t oe = __shfl_sync(kFull, orow, src);
-                        if (c0 + e < R) {
-                            const float val = (__uint_as_float(ohi[e]) - __uint_as_float(olo[e])) * ie;
-                            L.O[static_cast<size_t>(oe) * kHeadDim + dim] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                        }
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                                        __uint_as_float(o[2 * e + 1]) * inv);
+                        pk[e] = *reinterpret_cast<const uint32_t *>(&b2);
                     }
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cb + 32 * half);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
                 }
             }
             tc_fence_before();
