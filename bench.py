@@ -249,6 +249,20 @@ def oracle_sample(inp, wl, W, g, target_s: float):
 # arms
 # ------------------------------------------------------------------------------------------
 
+def rank_max(x: float, dist_mod, device) -> float:
+    """The largest x over the ranks of the process group: a job's time is its slowest rank's."""
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput in units of 1e12 per second: every rank processes units_per_rank
+    (weak scaling), and the job takes ms."""
+    return units_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -367,11 +381,9 @@ def run_ours(args):
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = float(sum(step_ms))
     if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = rank_max(total_ms, dist, dev)
     ms_per_step = total_ms / K
-    value = uflops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_rate(uflops, world, ms_per_step)
 
     # ---- end to end through the public API, host buffers ----
     e2e = None
@@ -407,10 +419,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / ne
         if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": uflops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s (useful)",
+            e2e_ms = rank_max(e2e_ms, dist, dev)
+        e2e = {"value": job_rate(uflops, world, e2e_ms), "unit": "TFLOP/s (useful)",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
