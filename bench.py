@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave out the per-configuration runs of the measurement plan")
+    ap.add_argument("--sweep-steps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -89,6 +92,31 @@ def group_work(gh: dict, G: int):
     rows = gh["gsize"].astype(np.int64) * G
     exec_flops = float((usize * rows).sum()) * PAGE * D * 4
     return union_bytes, exec_flops
+
+
+# Tensor-core work the pipelined kernel (tiles of <= 64 rows) issues per union page of a group,
+# whatever the group's row count R:
+#   S = Q K^T: two E4M3 parts of Q (K-concatenated), M = 64 rows (the tile, zero-padded), N = 64
+#     keys, K = 2 x 128 -> 2 * 64 * 64 * 256 FLOP.  An M = 64 product takes as long as an
+#     M = 128 one, so its tensor time is that of 2 * 128 * 64 * 256 FLOP at the E4M3 rate.
+#   O += P V: P_hi and P_lo stacked as one M = 128 operand, N = 128 dims, K = 64 keys
+#     -> 2 * 128 * 128 * 64 FLOP at the f16 rate.
+S_ISSUED_PER_PAGE = 2 * 64 * 64 * 256
+S_TIME_EQUIV_PER_PAGE = 2 * 128 * 64 * 256
+PV_ISSUED_PER_PAGE = 2 * 128 * 128 * 64
+FP8_OVER_BF16 = 2.0   # nominal dense E4M3 : bf16 throughput ratio of the tensor cores
+
+
+def issued_work(gh: dict):
+    """(issued tensor FLOPs, seconds those products need at the peaks, as a function of the
+    bf16 peak in TFLOP/s) of one pw_attn launch of the pipelined kernel."""
+    pages = float(np.diff(gh["union_off"]).astype(np.int64).sum())
+    issued = pages * (S_ISSUED_PER_PAGE + PV_ISSUED_PER_PAGE)
+
+    def seconds_at_peak(bf16_tflops: float) -> float:
+        return pages * (S_TIME_EQUIV_PER_PAGE / (FP8_OVER_BF16 * bf16_tflops * 1e12) +
+                        PV_ISSUED_PER_PAGE / (bf16_tflops * 1e12))
+    return issued, seconds_at_peak
 
 
 def source_hash(*paths) -> str:
@@ -166,12 +194,13 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, window=None):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = self.lines
-        if self.window is not None:
-            inside = [x for x in lines if self.window[0] <= x[0] <= self.window[1]]
+        lines = list(self.lines)
+        window = window if window is not None else self.window
+        if window is not None:
+            inside = [x for x in lines if window[0] <= x[0] <= window[1]]
             lines = inside if inside else lines
         for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -197,8 +226,9 @@ class ClockSampler:
 
 def oracle_sample(inp, wl, W, g, target_s: float):
     """Time the oracle on a bounded sample: the full grouping plus the attention of the rows
-    of the first groups of every kv head, grown until about target_s of CPU time.  Returns
-    (useful TFLOP/s of the oracle, threads, description, oracle ms per complete call)."""
+    of random groups, grown until about target_s of CPU time.  Returns (useful TFLOP/s of the
+    oracle, threads, description, estimated oracle ms of one complete call (extrapolated from
+    the sample), measured wall ms of the sample)."""
     from oracle import oracle
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
@@ -239,10 +269,11 @@ def oracle_sample(inp, wl, W, g, target_s: float):
     t_sample = t_attn + t_group * frac
     rate = flops_done / t_sample / 1e12
     full_ms = (t_group + t_attn / max(frac, 1e-12)) * 1e3
+    wall_ms = (t_group + t_attn) * 1e3
     desc = (f"full oracle grouping ({t_group:.2f} s) + oracle attention of all rows of "
             f"{sample_groups} random groups of {n_groups} ({frac * 100:.2f}% of the work, "
             f"{t_attn:.1f} s); grouping time apportioned by that fraction")
-    return rate, threads, desc, full_ms
+    return rate, threads, desc, full_ms, wall_ms
 
 
 # ------------------------------------------------------------------------------------------
@@ -274,16 +305,21 @@ def run_reference(args):
     per_step = max(args.cpu_seconds / max(args.steps, 1), 2.0)
     for _ in range(args.warmup):
         oracle_sample(inp, wl, args.W, args.g, 0.5)
-    rates, threads, desc, full_ms = [], 0, "", []
+    rates, threads, desc, full_ms, wall_ms = [], 0, "", [], []
     for _ in range(args.steps):
-        r, threads, desc, fm = oracle_sample(inp, wl, args.W, args.g, per_step)
+        r, threads, desc, fm, wm = oracle_sample(inp, wl, args.W, args.g, per_step)
         rates.append(r)
         full_ms.append(fm)
+        wall_ms.append(wm)
     value = statistics.median(rates)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s (useful)",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": statistics.median(full_ms), "higher_is_better": True,
+        # a step is one bounded sample of the workload (see cpu_baseline.sample): its measured
+        # wall time; the time of one whole call is an extrapolation, reported separately
+        "ms_per_step": statistics.median(wall_ms),
+        "full_call_ms_estimate": statistics.median(full_ms),
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, args),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s (useful)", "cores": threads,
@@ -301,6 +337,146 @@ def config_of(wl, args):
             "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "kmax": wl.kmax, "g": args.g, "W": args.W,
             "l2": "flushed (256 MiB write) before every timed step, outside the timed events",
             "parallelism": f"independent replicas x{args.gpus} (weak)"}
+
+
+class Timed:
+    """One configuration on the device: its inputs, group buffers and output, and the device
+    timing of complete calls (pw_group then pw_attn on the current stream, CUDA events)."""
+
+    def __init__(self, wl, W, g, dev, inp=None):
+        import torch
+        from dynamic_sparse_attention_pw_b200 import api, synth
+        self.api, self.wl, self.W, self.g = api, wl, W, g
+        self.inp = inp if inp is not None else synth.make_inputs(wl)
+        self.d = api.device_inputs(self.inp, dev)
+        self.status = api.new_status(dev)
+        self.groups = api.Groups.allocate(wl.T, wl.Hkv, self.inp["cu_seqlens"], wl.kmax, W, g, dev)
+        self.O = torch.empty_like(self.d["Q"])
+        self.stream = torch.cuda.current_stream()
+
+    def group(self):
+        d = self.d
+        self.api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], self.W, self.g,
+                          groups=self.groups, status=self.status)
+
+    def attn(self):
+        d = self.d
+        self.api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
+                         self.groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=self.O,
+                         status=self.status)
+
+    def run(self, steps, flush, warmup=3):
+        """Warm-up calls, then `steps` timed calls with L2 flushed before each (outside the
+        events), then up to 10 calls with L2 left warm.  Returns per-call (group, attn,
+        complete) ms lists, the warm-L2 list and the host window of the timed calls."""
+        import torch
+        for _ in range(warmup):
+            flush.fill_(1)
+            self.group()
+            self.attn()
+        torch.cuda.synchronize()
+        self.api.check_status(self.status, f"{self.wl.name} warm-up")
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        t0 = time.monotonic()
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(self.stream)
+            self.group()
+            ev[i][1].record(self.stream)
+            self.attn()
+            ev[i][2].record(self.stream)
+        torch.cuda.synchronize()
+        window = (t0, time.monotonic())
+        wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(steps, 10))]
+        for e in wev:
+            e[0].record(self.stream)
+            self.group()
+            self.attn()
+            e[1].record(self.stream)
+        torch.cuda.synchronize()
+        self.api.check_status(self.status, f"{self.wl.name} timed calls")
+        group_ms = [e[0].elapsed_time(e[1]) for e in ev]
+        attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+        warm_ms = [e[0].elapsed_time(e[1]) for e in wev]
+        return group_ms, attn_ms, step_ms, warm_ms, window
+
+    def work(self):
+        gh = self.groups.to_host()
+        union_bytes, exec_flops = group_work(gh, self.wl.G)
+        issued, at_peak = issued_work(gh)
+        usize = np.diff(gh["union_off"])
+        return {"gh": gh, "union_bytes": union_bytes, "exec_flops": exec_flops,
+                "issued_flops": issued, "tensor_seconds_at_peak": at_peak,
+                "useful_flops": useful_flops(self.inp, self.wl.Hq), "usize": usize}
+
+
+def breakdown(wk, group_ms, attn_ms, step_ms, warm_ms, hbm, bf16):
+    attn_mean = statistics.mean(attn_ms)
+    call_mean = statistics.mean(step_ms)
+    roof_ms = max(wk["union_bytes"] / (hbm * 1e9), wk["exec_flops"] / (bf16 * 1e12)) * 1e3
+    usize = wk["usize"]
+    return {
+        "group_ms": statistics.mean(group_ms), "attn_ms": attn_mean,
+        "group_ms_median": statistics.median(group_ms), "attn_ms_median": statistics.median(attn_ms),
+        "complete_call_ms": call_mean,
+        "complete_call_ms_median": statistics.median(step_ms),
+        "complete_call_ms_warm_l2_median": statistics.median(warm_ms),
+        "roofline_ms": roof_ms, "complete_call_frac_of_roofline": roof_ms / call_mean,
+        "attn_frac_of_roofline": roof_ms / attn_mean,
+        "union_pages_mean": float(usize.mean()) if usize.size else 0.0,
+        "union_pages_max": int(usize.max()) if usize.size else 0,
+        "n_groups": int(wk["gh"]["n_groups"]),
+        "useful_tflop": wk["useful_flops"] / 1e12,
+        "executed_tflop_algorithmic": wk["exec_flops"] / 1e12,
+        "useful_over_executed": wk["useful_flops"] / wk["exec_flops"] if wk["exec_flops"] else None,
+        "issued_tflop": wk["issued_flops"] / 1e12,
+        "useful_over_issued": wk["useful_flops"] / wk["issued_flops"] if wk["issued_flops"] else None,
+        "tensor_frac_issued_at_peak": wk["tensor_seconds_at_peak"](bf16) / (attn_mean * 1e-3),
+        "useful_tflops": wk["useful_flops"] / (call_mean * 1e-3) / 1e12,
+    }
+
+
+# The per-configuration runs of the measurement plan: the 64K workload swept over W, the 32K
+# workload grouped three ways (contiguous W = g, regrouped W = 128, one query per group), and the
+# remaining workloads at their own W.
+SWEEP = [(4, 32, 8), (4, 64, 8), (4, 256, 8), (3, 8, 8), (3, 128, 8), (3, 128, 1),
+         (1, 32, 8), (2, 64, 8), (5, 128, 8)]
+
+
+def run_sweep(args, dev, flush, clocks, hbm, bf16, head_inp):
+    """One entry per SWEEP configuration (the headline configuration is the line itself)."""
+    import torch
+    from dynamic_sparse_attention_pw_b200 import synth
+    out = []
+    inputs = {args.workload: head_inp}
+    for cfg, W, g in SWEEP:
+        if (cfg, W, g) == (args.workload, args.W, args.g):
+            continue
+        wl = synth.WORKLOADS[cfg].with_(W=W, g=g)
+        if cfg not in inputs:
+            inputs = {cfg: synth.make_inputs(synth.WORKLOADS[cfg])}
+        t = Timed(wl, W, g, dev, inp=inputs[cfg])
+        gm, am, sm_, wm, window = t.run(args.sweep_steps, flush)
+        wk = t.work()
+        bd = breakdown(wk, gm, am, sm_, wm, hbm, bf16)
+        achieved = wk["union_bytes"] / (bd["attn_ms"] * 1e-3) / 1e9
+        entry = {"workload": wl.name, "T": wl.T, "W": W, "g": g, "steps": args.sweep_steps,
+                 "union_pages_mean": bd["union_pages_mean"], "union_pages_max": bd["union_pages_max"],
+                 "group_ms": bd["group_ms"], "attn_ms": bd["attn_ms"],
+                 "complete_call_ms": bd["complete_call_ms"],
+                 "complete_call_ms_warm_l2_median": bd["complete_call_ms_warm_l2_median"],
+                 "useful_tflops": bd["useful_tflops"],
+                 "attn_frac_of_roofline": bd["attn_frac_of_roofline"],
+                 "union_byte_rate_gbs": achieved,
+                 "useful_over_issued": bd["useful_over_issued"],
+                 "tensor_frac_issued_at_peak": bd["tensor_frac_issued_at_peak"],
+                 "clocks": clocks.summary(window)}
+        out.append(entry)
+        del t
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -321,76 +497,32 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
 
     wl = synth.WORKLOADS[args.workload].with_(W=args.W, g=args.g)
-    inp = synth.make_inputs(wl)
-    d = api.device_inputs(inp, dev)
-    status = api.new_status(dev)
-    groups = api.Groups.allocate(wl.T, wl.Hkv, inp["cu_seqlens"], wl.kmax, args.W, args.g, dev)
-    O = torch.empty_like(d["Q"])
+    head = Timed(wl, args.W, args.g, dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], args.W, args.g,
-                     groups=groups, status=status)
-        api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
-                    groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=O, status=status)
-
     clocks = ClockSampler(dev.index).__enter__()
-    for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
-        step()
-    torch.cuda.synchronize()
-    api.check_status(status, "bench warm-up")
-    gh = groups.to_host()
-    union_bytes, exec_flops = group_work(gh, wl.G)
-    uflops = useful_flops(inp, wl.Hq)
-    usize = np.diff(gh["union_off"])
-
-    # ---- device-timed region ----
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    # ---- device-timed region (the same calls on every rank, then the slowest rank's time) ----
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    t_start = time.monotonic()
-    for i in range(K):
-        flush.fill_(i & 0xFF)
-        ev[i][0].record(stream)
-        api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], args.W, args.g,
-                     groups=groups, status=status)
-        ev[i][1].record(stream)
-        api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"],
-                    groups, d["k_scale"], d["v_scale"], d["sm_scale"], O=O, status=status)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    clocks.mark(t_start, time.monotonic())
-    clocks.__exit__(None, None, None)
-    # secondary figure: the same calls with L2 left warm (no flush between them)
-    wev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(K, 10))]
-    for e in wev:
-        e[0].record(stream)
-        step()
-        e[1].record(stream)
-    torch.cuda.synchronize()
-    warm_ms = [e[0].elapsed_time(e[1]) for e in wev]
+    group_ms, attn_ms, step_ms, warm_ms, window = head.run(K, flush, warmup=max(args.warmup, 3))
+    clocks.mark(*window)
     if world > 1:
         dist.barrier()
-    api.check_status(status, "bench timed region")
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    group_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = float(sum(step_ms))
     if world > 1:
         total_ms = rank_max(total_ms, dist, dev)
     ms_per_step = total_ms / K
-    value = job_rate(uflops, world, ms_per_step)
+    wk = head.work()
+    value = job_rate(wk["useful_flops"], world, ms_per_step)
 
     # ---- end to end through the public API, host buffers ----
     e2e = None
+    d = head.d
     if not args.no_e2e:
         pin = {k: d[k].cpu().pin_memory() for k in ("Q", "K_pages", "V_pages", "page_table",
                                                      "sel_pages", "cu_seqlens")}
-        out_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        out_host = torch.empty(head.O.shape, dtype=head.O.dtype).pin_memory()
         dev_bufs = {k: torch.empty_like(d[k]) for k in pin}
         h2d = int(sum(v.numel() * v.element_size() for v in pin.values()))
         d2h = int(out_host.numel() * out_host.element_size())
@@ -401,8 +533,8 @@ def run_ours(args):
             api.prefill(dev_bufs["Q"], dev_bufs["K_pages"], dev_bufs["V_pages"],
                         dev_bufs["page_table"], dev_bufs["sel_pages"], dev_bufs["cu_seqlens"],
                         d["cu_seqlens_host"], args.W, args.g, d["k_scale"], d["v_scale"],
-                        d["sm_scale"], groups=groups, O=O, status=status)
-            out_host.copy_(O, non_blocking=True)
+                        d["sm_scale"], groups=head.groups, O=head.O, status=head.status)
+            out_host.copy_(head.O, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -412,30 +544,36 @@ def run_ours(args):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         ne = max(2, min(K, 5))
-        e0.record(stream)
+        e0.record(head.stream)
         for _ in range(ne):
             e2e_step()
-        e1.record(stream)
+        e1.record(head.stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / ne
         if world > 1:
             e2e_ms = rank_max(e2e_ms, dist, dev)
-        e2e = {"value": job_rate(uflops, world, e2e_ms), "unit": "TFLOP/s (useful)",
+        e2e = {"value": job_rate(wk["useful_flops"], world, e2e_ms), "unit": "TFLOP/s (useful)",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
+        clocks.__exit__(None, None, None)
         if world > 1:
             dist.destroy_process_group()
         return 0
 
     hbm, bf16, src = peaks()
-    attn_mean = statistics.mean(attn_ms)
-    achieved = union_bytes / (attn_mean * 1e-3) / 1e9
+    sweep = None
+    if not args.no_sweep and world == 1:
+        sweep = run_sweep(args, dev, flush, clocks, hbm, bf16, head.inp)
+    clocks.__exit__(None, None, None)
+
+    bd = breakdown(wk, group_ms, attn_ms, step_ms, warm_ms, hbm, bf16)
+    attn_mean = bd["attn_ms"]
+    achieved = wk["union_bytes"] / (attn_mean * 1e-3) / 1e9
     ksrc = os.path.join(ROOT, "dynamic_sparse_attention_pw_b200", "csrc")
     khash = source_hash(*(os.path.join(ksrc, f) for f in
                           ("pw_attn.cu", "pw_attn_ws.cu", "pw_attn_common.cuh", "pw_sm100.cuh")))
     kname = "k_union_attn_ws" if args.g * wl.G <= 64 else "k_union_attn"
-    roof_ms = max(union_bytes / (hbm * 1e9), exec_flops / (bf16 * 1e12)) * 1e3
     line = {
         "metric": METRIC,
         "value": value,
@@ -455,30 +593,22 @@ def run_ours(args):
             "frac": achieved / hbm, "traffic": traffic_from_profile(khash),
             "kernel": kname, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)"
             if src == "measured" else "fallback 6650 GB/s",
-            "algorithmic_bytes_per_launch": union_bytes,
+            "achieved_is": "union-byte rate: the K and V pages of every group's union counted once "
+                           "per group, over the kernel's time; pages shared by nearby groups come "
+                           "from L2, so DRAM moves far fewer bytes (traffic)",
+            "algorithmic_bytes_per_launch": wk["union_bytes"],
             "kernel_ms": attn_mean,
         },
-        "breakdown": {
-            "group_ms": statistics.mean(group_ms), "attn_ms": attn_mean,
-            "group_ms_median": statistics.median(group_ms), "attn_ms_median": statistics.median(attn_ms),
-            "complete_call_ms_median": statistics.median(step_ms),
-            "complete_call_ms_warm_l2_median": statistics.median(warm_ms),
-            "complete_call_ms": ms_per_step,
-            "roofline_ms": roof_ms, "complete_call_frac_of_roofline": roof_ms / ms_per_step,
-            "attn_frac_of_roofline": roof_ms / attn_mean,
-            "union_pages_mean": float(usize.mean()), "union_pages_max": int(usize.max()),
-            "n_groups": int(gh["n_groups"]),
-            "useful_tflop": uflops / 1e12, "executed_tflop_algorithmic": exec_flops / 1e12,
-            "useful_over_executed": uflops / exec_flops,
-            "tensor_frac_executed": exec_flops / (attn_mean * 1e-3) / (bf16 * 1e12),
-        },
+        "breakdown": bd,
         "clocks": clocks.summary(),
         "gpu_launches": 5 * K,
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if sweep is not None:
+        line["sweep"] = sweep
     if not args.no_cpu_baseline and world == 1:
-        rate, threads, desc, _ = oracle_sample(inp, wl, args.W, args.g, args.cpu_seconds)
+        rate, threads, desc, _, _ = oracle_sample(head.inp, wl, args.W, args.g, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s (useful)", "cores": threads,
                                 "kind": "oracle", "sample": desc}
     print(json.dumps(line))

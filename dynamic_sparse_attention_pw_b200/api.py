@@ -131,16 +131,30 @@ def pw_attn(Q: torch.Tensor, K_pages: torch.Tensor, V_pages: torch.Tensor,
             page_table: torch.Tensor, cu_seqlens: torch.Tensor, groups: Groups,
             k_scale: float = 1.0, v_scale: float = 1.0, sm_scale: float | None = None,
             O: torch.Tensor | None = None, status: torch.Tensor | None = None,
-            stream=None) -> torch.Tensor:
+            stream=None, cu_seqlens_host=None) -> torch.Tensor:
     """ID-aware union attention (include/pw.h, pw_attn).  Q bf16 [T, Hq, 128];
-    K_pages/V_pages uint8 E4M3 codes [n_phys, Hkv, 64, 128]; returns O bf16 [T, Hq, 128]."""
+    K_pages/V_pages uint8 E4M3 codes [n_phys, Hkv, 64, 128]; page_table int32 [B, max_pages]
+    with B = len(cu_seqlens) - 1; returns O bf16 [T, Hq, 128].  With cu_seqlens_host (a host
+    copy of cu_seqlens) the page table's width is checked against the longest sequence."""
     L = _lib.load()
     T, Hq, D = Q.shape
     assert Q.is_cuda and Q.dtype == torch.bfloat16 and Q.is_contiguous() and D == 128
+    for t in (K_pages, V_pages, page_table, cu_seqlens):
+        assert t.is_cuda and t.device == Q.device and t.is_contiguous()
     assert K_pages.dtype == torch.uint8 and V_pages.dtype == torch.uint8
-    assert K_pages.is_contiguous() and V_pages.is_contiguous()
+    assert K_pages.dim() == 4 and tuple(K_pages.shape[2:]) == (64, 128)
+    assert K_pages.shape == V_pages.shape
     n_phys, Hkv = K_pages.shape[0], K_pages.shape[1]
-    assert page_table.dtype == torch.int32 and page_table.is_contiguous()
+    assert Hq % Hkv == 0
+    assert cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1
+    B = cu_seqlens.numel() - 1
+    assert page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.shape[0] == B
+    assert groups.bits.numel() >= T * Hkv * groups.words
+    if cu_seqlens_host is not None:
+        cu = _host_cu(cu_seqlens_host)
+        assert len(cu) == B + 1 and int(cu[-1]) == T
+        max_len = int(np.max(np.diff(cu))) if B > 0 else 0
+        assert page_table.shape[1] >= (max_len + 63) // 64, "page table narrower than a sequence"
     if sm_scale is None:
         sm_scale = 1.0 / float(np.sqrt(D))
     if O is None:
@@ -149,7 +163,7 @@ def pw_attn(Q: torch.Tensor, K_pages: torch.Tensor, V_pages: torch.Tensor,
         status = new_status(Q.device)
     st = groups.struct()
     _check(L.pw_attn(_ptr(Q), _ptr(K_pages), _ptr(V_pages), _ptr(page_table),
-                     page_table.shape[1], n_phys, _ptr(cu_seqlens), page_table.shape[0], T, Hq,
+                     page_table.shape[1], n_phys, _ptr(cu_seqlens), B, T, Hq,
                      Hkv, float(k_scale), float(v_scale), float(sm_scale), C.byref(st), _ptr(O),
                      _ptr(status), _stream(stream)), "pw_attn")
     return O
@@ -164,7 +178,7 @@ def prefill(Q, K_pages, V_pages, page_table, sel_pages, cu_seqlens, cu_seqlens_h
     groups = pw_group(sel_pages, cu_seqlens, cu_seqlens_host, W, g, groups=groups, status=status,
                       stream=stream)
     O = pw_attn(Q, K_pages, V_pages, page_table, cu_seqlens, groups, k_scale, v_scale, sm_scale,
-                O=O, status=status, stream=stream)
+                O=O, status=status, stream=stream, cu_seqlens_host=cu_seqlens_host)
     return O, groups
 
 

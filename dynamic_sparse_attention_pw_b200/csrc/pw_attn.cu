@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
     const int u0 = L.union_off[gi];
     const int nU = L.union_off[gi + 1] - u0;
     const uint32_t kIdescPV = idesc_bf16_f32(128, Npad, true, false);
+    if (!group_scalars_ok(L, b, h, L.gsize[gi], nU))
+        return;
+    const int32_t cu_b = L.cu[b], cu_e = L.cu[b + 1];
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s)
@@ -116,6 +119,10 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
             const int mi = i / L.G;
             tok = L.qids[gi * L.g + mi];
             hq = h * L.G + (i - mi * L.G);
+            if (tok < cu_b || tok >= cu_e) { // a member outside the group's sequence
+                set_status(L.status, PW_ERR_INVALID_ARG);
+                tok = cu_b;
+            }
         }
         sm.row_tok[i] = tok;
         sm.row_hq[i] = hq;
@@ -123,13 +130,8 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
     }
     for (int i = tid; i < nU && i < kUnionCache; i += NT) {
         const int pg = L.union_pages[u0 + i];
-        int phys = L.page_table[static_cast<size_t>(b) * L.max_pages + pg];
-        if (phys < 0 || phys >= L.n_phys) {
-            set_status(L.status, PW_ERR_INVALID_ARG);
-            phys = 0;
-        }
         sm.upage[i] = pg;
-        sm.uphys[i] = phys;
+        sm.uphys[i] = phys_page(L, b, pg);
     }
     if (tid == 0)
         sm.rescale = 0;
@@ -175,11 +177,7 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
         if (i < kUnionCache) {
             phys = sm.uphys[i];
         } else {
-            phys = L.page_table[static_cast<size_t>(b) * L.max_pages + L.union_pages[u0 + i]];
-            if (phys < 0 || phys >= L.n_phys) {
-                set_status(L.status, PW_ERR_INVALID_ARG);
-                phys = 0;
-            }
+            phys = phys_page(L, b, L.union_pages[u0 + i]);
         }
         const size_t off = (static_cast<size_t>(phys) * L.Hkv + h) * kPageBytes;
         mbar_arrive_expect_tx(&sm.tma_bar[s], 2 * kPageBytes);
@@ -199,7 +197,7 @@ __global__ void __launch_bounds__(128 * RB, (RB == 1) ? 2 : 1) k_union_attn(cons
         const int s = i % kStages;
         const int pg = page_of(i);
         // membership word of my row for this page, fetched now so the decode hides its latency
-        const uint32_t word = row_valid ? __ldg(bitrow + (pg >> 5)) : 0u;
+        const uint32_t word = row_valid ? __ldg(bitrow + page_word(L, pg)) : 0u;
         bool ok = true;
         if (mma_pending) { // previous O^T += V^T P^T: frees v and p, settles O^T
             ok = mbar_wait(&sm.mma_bar, mma_phase);

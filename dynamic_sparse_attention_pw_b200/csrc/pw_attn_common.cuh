@@ -6,12 +6,50 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "pw_internal.h"
+#include "pw_sm100.cuh"
+
 namespace pw {
 namespace attn {
 
 constexpr int kPageBytes = 64 * 128; // one kv head's page, E4M3
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Physical slot of logical page pg of sequence b through the page table.  A page outside the
+// table's row (a table narrower than the sequence) or a slot outside [0, n_phys) records
+// PW_ERR_INVALID_ARG and gives slot 0, so that nothing is read outside the caller's buffers.
+__device__ __forceinline__ int phys_page(const AttnLaunch &L, int b, int pg)
+{
+    if (pg < 0 || pg >= L.max_pages) {
+        set_status(L.status, PW_ERR_INVALID_ARG);
+        return 0;
+    }
+    const int phys = L.page_table[static_cast<size_t>(b) * L.max_pages + pg];
+    if (phys < 0 || phys >= L.n_phys) {
+        set_status(L.status, PW_ERR_INVALID_ARG);
+        return 0;
+    }
+    return phys;
+}
+
+// Word of a membership bitset row holding page pg's bit, kept inside the row for any pg.
+__device__ __forceinline__ uint32_t page_word(const AttnLaunch &L, int pg)
+{
+    const uint32_t w = static_cast<uint32_t>(pg) >> 5;
+    return w < static_cast<uint32_t>(L.words) ? w : static_cast<uint32_t>(L.words - 1);
+}
+
+// Whether the scalars of group gi's record address only what the launch owns: sequence and kv
+// head in range, 1..g members and a non-negative union length.  (The member tokens are checked
+// against the sequence by the caller.)  A bad record is recorded as PW_ERR_INVALID_ARG.
+__device__ __forceinline__ bool group_scalars_ok(const AttnLaunch &L, int b, int h, int gsz, int nU)
+{
+    const bool ok = b >= 0 && b < L.B && h >= 0 && h < L.Hkv && gsz >= 1 && gsz <= L.g && nU >= 0;
+    if (!ok)
+        set_status(L.status, PW_ERR_INVALID_ARG);
+    return ok;
+}
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled operand tile
 // (rows of 128 bytes, chunks XOR-swizzled by row % 8, 8-row atoms at 1024 bytes).

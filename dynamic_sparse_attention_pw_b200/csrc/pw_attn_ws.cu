@@ -12,11 +12,12 @@
 // O += P V runs on f16 operands with P read from TMEM: P split into f16 hi + lo parts, both
 // multiplied into the one accumulator, and V decoded exactly (E4M3 is a subset of f16).
 //
-// One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  Its warps:
-//   warps 0-3    decode   E4M3 V pages -> f16 operand tiles
-//   warps 4-11   softmax  S -> P for each step of one or two pages (four threads per row,
-//                         16 keys of each page each), written back to TMEM over the S it came
-//                         from; lazy O rescale (out of line); per-row sums of each group
+// One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  A step is one or
+// two union pages of a group.  Its warps:
+//   warps 0-3    decode   E4M3 V pages -> f16 operand tiles, one step at a time
+//   warps 4-11   softmax  S -> P for each step (four threads per row, 16 keys of each page each;
+//                         both pages' scores in one TMEM round trip), written back to TMEM over
+//                         the S it came from; lazy O rescale (out of line); per-row sums
 //   warps 12-15  epilogue Q tile of the next group (scaled, split into two E4M3 parts) while
 //                         the current one runs, then O of the finished group -> bf16 rows of O
 //                         (one warp per TMEM lane quadrant)
@@ -24,19 +25,20 @@
 //                         words, first page ids), the next group's Q rows by TMA, and the union
 //                         pages: K through a tensor map with the 128-byte swizzle the MMA reads,
 //                         V by bulk copy
-//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O += P V for the
-//                         pages of step n - 1
+//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O += P V for step
+//                         n - 1
 // Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
 // its scheduler delays its waits and issues.  Compact code on purpose too: five roles run
-// different code on each scheduler, so cold paths stay out of line or rolled and each role's
-// loop calls its steps from one place, leaving the instruction cache to the hot loops.
+// different code on each scheduler, and on most SMs the kernel slows down in proportion to its
+// code size, so cold paths stay out of line or rolled and each role's loop calls each of its
+// steps from one place.
 // TMEM holds two S buffers and two O buffers (M = 64 layout: row r at lane 32 (r / 16) + r % 16).
 // The P of a step replaces its S in place, as the A operand of the products (keys 2j and 2j + 1
-// of a 16-key block packed in column j: P_hi in a block's first 8 columns, P_lo in the next 8);
-// S two steps later overwrites it only after those products are done.  A K stage is free once S
-// is done, a V stage once it is decoded, an f16 V slot once the product is done.  O is
-// double-buffered across groups.  Every hand-off is an mbarrier; every wait is bounded and, when
-// it runs out, sets an abort flag that releases the other roles.
+// of a 16-key block packed in column j: P_hi in a block's first 8 columns, P_lo in the next 8).
+// Hand-offs per step, all mbarriers: S done (also frees the step's K stage pair), P written, V
+// tiles decoded, products done (frees the S/P buffer for S two steps later and the V step slot
+// for the tiles two steps later).  O is double-buffered across groups.  Every wait is bounded
+// and, when it runs out, sets an abort flag that releases the other roles.
 #include <cstdint>
 #include <cuda.h> // CUtensorMap and its enums (the encoder itself is fetched at run time)
 #include <cuda_bf16.h>
@@ -52,10 +54,9 @@ namespace {
 
 using namespace attn;
 
-constexpr int kNKP = 2;       // E4M3 K stage pairs (one S step each)
-constexpr int kNSV = 3;       // E4M3 V page stages
+constexpr int kNKP = 2;       // E4M3 K stage pairs (one S step each), paired with the S buffers
+constexpr int kNSV = 4;       // E4M3 V page stages
 constexpr int kNJ = 3;        // group records in flight
-constexpr int kNV = 3;        // f16 V slots
 constexpr int kDecThreads = 128;
 constexpr int kSmThreads = 256;
 constexpr int kEpiThreads = 128;
@@ -64,6 +65,7 @@ constexpr int kWarpSm0 = kDecThreads / 32, kWarpEpi0 = kWarpSm0 + 8, kWarpLoad =
 constexpr int kThreads = 32 * (kWarpMma + 1);
 static_assert(kWarpSm0 % 4 == 0, "softmax warp w must sit in TMEM lane quadrant w % 4");
 static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
+static_assert(kNKP == 2, "a K stage pair is freed by the S completion of its S buffer");
 constexpr uint32_t kTmemCols = 512; // S / P [0..1] at columns 0 / 128, O[0..1] at 256 / 384
 constexpr uint32_t kColS = 128;     // one S step: two pages of 64 keys
 constexpr uint32_t kColO = 256;
@@ -80,8 +82,8 @@ struct GroupJob {
 };
 
 struct __align__(1024) WsSmem {
-    uint8_t q[2][2][64 * 128];   // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
-    uint8_t v[kNV][2][64 * 128]; // [slot][dim-block][64 keys][64 dims] f16, swizzled
+    uint8_t q[2][2][64 * 128];    // [Q buffer][part q1 / q2][64 rows][128 dims] E4M3, swizzled
+    uint8_t v[2][2][2][64 * 128]; // [step slot][page of the step][dim-block][64 keys][64 dims] f16, swizzled
     // E4M3 K pages, 128-byte swizzled by the tensor copy; the two pages of a step sit in one
     // pair, so that they form one 128-row operand
     uint8_t stage_k[kNKP][2][kPageBytes];
@@ -92,11 +94,14 @@ struct __align__(1024) WsSmem {
     float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
     uint64_t job_full[kNJ], job_empty[kNJ];
     uint64_t qraw_full, qraw_empty;
-    uint64_t kst_full[kNKP], kst_empty[kNKP];
+    uint64_t kst_full[kNKP];
     uint64_t vst_full[kNSV], vst_empty[kNSV];
-    uint64_t v_full[kNV], v_empty[kNV]; // v_empty[i % kNV]: the product of page i is complete
-    uint64_t s_done[2];                 // s_done[n % 2]: S of step n complete
-    uint64_t pvs_done[2];               // pvs_done[n % 2]: the products of step n complete
+    uint64_t v_full[2];   // v_full[n % 2]: the f16 V tiles of step n decoded
+    // s_done[n % 2]: S of step n complete; this also frees S's K stage pair (pair n % 2)
+    uint64_t s_done[2];
+    // pvs_done[n % 2]: the products of step n complete; this frees S/P buffer n % 2 for S of
+    // step n + 2 and the V step slot n % 2 for the tiles of step n + 2
+    uint64_t pvs_done[2];
     uint64_t p_full[2];                 // p_full[n % 2]: P of both pages of step n written
     uint64_t q_full[2], q_empty[2];
     uint64_t o_full[2]; // last product of the group in O buffer b complete
@@ -286,33 +291,30 @@ __device__ __forceinline__ void split_q8(const uint4 v, float scale, uint2 &q1, 
     q2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
-// Largest of the first nq of 16 scores, sign-flipped when the log2-domain factor is negative.
-__device__ __forceinline__ float quarter_max(const uint32_t (&sv)[16], int nq, bool flip)
+// Largest of this thread's 16 scores of a page over its allowed keys (the first nq), -inf when
+// none is allowed.  Each thread takes the case of its own nq: a page not selected by the row's
+// query (nq = 0) costs nothing, a fully allowed one needs no predicates.
+__device__ __forceinline__ float page_max(const uint32_t (&sv)[16], int nq)
 {
+    if (nq == 0)
+        return -INFINITY;
+    if (nq == 16) {
+        float m0 = __uint_as_float(sv[0]), m1 = __uint_as_float(sv[1]);
+        float m2 = __uint_as_float(sv[2]), m3 = __uint_as_float(sv[3]);
+#pragma unroll
+        for (int e = 4; e < 16; e += 4) {
+            m0 = fmaxf(m0, __uint_as_float(sv[e]));
+            m1 = fmaxf(m1, __uint_as_float(sv[e + 1]));
+            m2 = fmaxf(m2, __uint_as_float(sv[e + 2]));
+            m3 = fmaxf(m3, __uint_as_float(sv[e + 3]));
+        }
+        return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+    }
     float lm = -INFINITY;
-    if (__all_sync(0xFFFFFFFFu, nq == 16)) { // every key allowed: a tree, no predicates
-        float m[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            m[e] = flip ? -__uint_as_float(sv[e]) : __uint_as_float(sv[e]);
-#pragma unroll
-        for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-            for (int e = 0; e < w; ++e)
-                m[e] = fmaxf(m[e], m[e + w]);
-        return m[0];
-    }
-    if (!flip) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            if (e < nq)
-                lm = fmaxf(lm, __uint_as_float(sv[e]));
-    } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            if (e < nq)
-                lm = fmaxf(lm, -__uint_as_float(sv[e]));
-    }
+    for (int e = 0; e < 16; ++e)
+        if (e < nq)
+            lm = fmaxf(lm, __uint_as_float(sv[e]));
     return lm;
 }
 
@@ -370,9 +372,9 @@ __device__ __forceinline__ void tmem_st_16x32bx2_x32s(uint32_t taddr, const uint
                  : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem] with kind::f16: A is read from TMEM (for M = 64, row r at lane
-// 32 (r / 16) + r % 16, keys 2j and 2j + 1 packed in column j), B from a shared-memory
-// descriptor.
+// D[tmem] (+)= A[tmem] * B[smem] with kind::f16: A is read from TMEM (row r at lane r for M = 128;
+// for M = 64 at lane 32 (r / 16) + r % 16; keys 2j and 2j + 1 packed in column j), B from a
+// shared-memory descriptor.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                            uint32_t idesc, uint32_t accumulate)
 {
@@ -383,16 +385,27 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
                  : "memory");
 }
 
-// P of the 16 keys of one row that this thread read from TMEM at s_addr (the first nq allowed,
-// the rest 0), written back over those columns as the A operand of O += P V: P_hi in the first
-// 8 columns, P_lo in the last 8 (for lanes 16-31 of the warp, 16 columns further on, as they were
-// read).  Returns the keys' sum.
-__device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float c, float negm,
-                                        uint32_t s_addr)
+// Wait for this thread's outstanding tcgen05.ld into two 16-register arrays (both routed through
+// the asm, so that no use of them is scheduled before the wait).
+__device__ __forceinline__ void tmem_ld_wait2x16(uint32_t (&a)[16], uint32_t (&b)[16])
 {
-    uint32_t hi[8], lo[8];
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]),
+                   "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]),
+                   "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(b[0]), "+r"(b[1]),
+                   "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
+                   "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]),
+                   "+r"(b[14]), "+r"(b[15])::"memory");
+}
+
+// P = 2^(s c + negm) of the 16 keys of one row that this thread read of one page (the first nq
+// allowed, the rest 0), split into f16 hi + lo parts (keys 2j, 2j + 1 in word j).  Returns the
+// keys' sum.  As in page_max, each thread takes the case of its own nq.
+__device__ __forceinline__ float p_page(const uint32_t (&sv)[16], int nq, float c, float negm,
+                                        uint32_t (&hi)[8], uint32_t (&lo)[8])
+{
     float sum = 0.f;
-    if (__all_sync(0xFFFFFFFFu, nq == 16)) {
+    if (nq == 16) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
@@ -400,6 +413,10 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             sum += p0 + p1;
             split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
+    } else if (nq == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            hi[e] = lo[e] = 0u;
     } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -409,27 +426,32 @@ __device__ __forceinline__ float emit_p(const uint32_t (&sv)[16], int nq, float 
             split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
     }
-    tmem_st_16x32bx2_x8(s_addr, hi);
-    tmem_st_16x32bx2_x8(s_addr + 8, lo);
     return sum;
+}
+
+// The hi/lo parts of one page's 16 keys of one row, written back over the 16 columns this thread
+// read them from (as the A operand of O += P V): P_hi in the first 8 columns, P_lo in the last 8
+// (for lanes 16-31 of the warp, 16 columns further on, as they were read).
+__device__ __forceinline__ void store_p(const uint32_t (&hi)[8], const uint32_t (&lo)[8], uint32_t p_addr)
+{
+    tmem_st_16x32bx2_x8(p_addr, hi);
+    tmem_st_16x32bx2_x8(p_addr + 8, lo);
 }
 
 // The softmax role's slow path, taken when some row's scores exceed its running max by more
 // than 2^8 (always at a group's first step): the row's four threads agree on its max and, when
-// a row's max rises, O[r, :] *= alpha[r] once every product issued so far (those of the pages up
-// to wait_to) has completed.  Kept out of line so that the common
-// path of the softmax loop stays small in the instruction cache.  Every thread of the role calls
-// it; the state comes back by value.
+// a row's max rises, O[r, :] *= alpha[r] once every product issued so far (those of the steps
+// before stp) has completed.  Kept out of line so that the common path of the softmax loop stays
+// small in the instruction cache.  Every thread of the role calls it; the state comes back by
+// value.
 struct SlowOut {
     float m_used, l_part;
-    uint32_t pv_done;
     bool ok;
 };
 
 __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, int hw, bool any, float lm,
                                                   float m_used, float l_part, bool first_step,
-                                                  uint32_t wait_to, uint32_t pv_done, bool sleader,
-                                                  uint32_t o_addr)
+                                                  uint32_t stp, bool sleader, uint32_t o_addr)
 {
     sm.qmax[row][qq] = any ? lm : -INFINITY;
     softmax_bar();
@@ -446,14 +468,13 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
     }
     // (at a group's first step no row has a max yet, so none rescales)
     if (!first_step && softmax_bar_or(rescale)) {
-        // v_empty[x % kNV] completes once per product of page x, and a parity wait is only
-        // unambiguous one phase ahead of what is known complete: step through the pages in order.
-        bool ok = true;
-        for (; pv_done <= wait_to && ok; ++pv_done)
-            if (sleader && !wait_bar(&sm.v_empty[pv_done % kNV], (pv_done / kNV) & 1u, &sm.abort_flag))
-                ok = false;
+        // pvs_done of step stp - 1 covers every product issued before it.  Its phase is
+        // unambiguous: S of this step was issued after the products of step stp - 2 had
+        // completed, and the products of step stp + 1 cannot have run yet.
+        const bool ok = !sleader ||
+                        wait_bar(&sm.pvs_done[(stp - 1) & 1u], ((stp - 1) >> 1) & 1u, &sm.abort_flag);
         if (softmax_bar_or(!ok))
-            return SlowOut{m_used, l_part, pv_done, false};
+            return SlowOut{m_used, l_part, false};
         // O[r, :] *= alpha[r]: the row sits in this warp's lanes, and its four threads take 32
         // head dimensions each (lanes 0-15 dims 64 hw .. 64 hw + 31, lanes 16-31 the next 32).
         tc_fence_after();
@@ -466,7 +487,7 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
         tmem_st_16x32bx2_x32s(o_addr + 64 * hw, o);
         tmem_st_wait();
     }
-    return SlowOut{m_used, l_part, pv_done, true};
+    return SlowOut{m_used, l_part, true};
 }
 
 // tmap_k: the K pages as a 2-D byte tensor [n_phys * Hkv * 64 rows][128], boxes of 64 x 128
@@ -493,19 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.qraw_full, 1);
         mbar_init(&sm.qraw_empty, kEpiThreads / 32);
-        for (int s = 0; s < kNKP; ++s) {
+        for (int s = 0; s < kNKP; ++s)
             mbar_init(&sm.kst_full[s], 1);
-            mbar_init(&sm.kst_empty[s], 1);
-        }
         for (int s = 0; s < kNSV; ++s) {
             mbar_init(&sm.vst_full[s], 1);
             mbar_init(&sm.vst_empty[s], kDecThreads / 32);
         }
-        for (int s = 0; s < kNV; ++s) {
-            mbar_init(&sm.v_full[s], kDecThreads / 32);
-            mbar_init(&sm.v_empty[s], 1);
-        }
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.v_full[s], kDecThreads / 32);
             mbar_init(&sm.s_done[s], 1);
             mbar_init(&sm.pvs_done[s], 1);
             mbar_init(&sm.p_full[s], kSmThreads / 32);
@@ -550,11 +566,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t w0_l, w1_l;   // lane l: its membership words of the first two union pages
         };
         // The next group with union pages, from gi on; groups without any get their zero rows.
+        // A record that would address outside the launch's buffers (sequence, head, size or a
+        // member token out of range) is skipped and recorded as PW_ERR_INVALID_ARG.
         auto next_group = [&](int64_t gi, GMeta &m) -> bool {
             for (; gi < L.n_groups; gi += gstep) {
                 const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
                 const int gsz = L.gsize[gi], R = gsz * L.G;
                 const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
+                if (!group_scalars_ok(L, b, h, gsz, nU))
+                    continue;
+                const int32_t cu_b = L.cu[b], cu_e = L.cu[b + 1];
+                const int32_t tok_l = lane < gsz ? L.qids[gi * L.g + lane] : cu_b;
+                if (!__all_sync(kFull, tok_l >= cu_b && tok_l < cu_e)) {
+                    if (lane == 0)
+                        set_status(L.status, PW_ERR_INVALID_ARG);
+                    continue;
+                }
                 if (nU == 0) {
                     for (int idx = lane; idx < R * 16; idx += 32) {
                         const int r = idx >> 4, c = idx & 15, mi = r / L.G;
@@ -572,15 +599,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m.R = R;
                 m.u0 = u0;
                 m.nU = nU;
-                m.tok_l = lane < gsz ? L.qids[gi * L.g + lane] : 0;
-                m.cu_b = L.cu[b];
+                m.tok_l = lane < gsz ? tok_l : 0;
+                m.cu_b = cu_b;
                 m.pg0 = L.union_pages[u0];
                 m.pg1 = nU > 1 ? L.union_pages[u0 + 1] : m.pg0;
                 m.pg2 = nU > 2 ? L.union_pages[u0 + 2] : m.pg0;
                 m.pg3 = nU > 3 ? L.union_pages[u0 + 3] : m.pg0;
                 const uint32_t *bitrow = L.bits + (static_cast<size_t>(m.tok_l) * L.Hkv + h) * L.words;
-                m.w0_l = lane < gsz ? __ldg(bitrow + (m.pg0 >> 5)) : 0u;
-                m.w1_l = lane < gsz ? __ldg(bitrow + (m.pg1 >> 5)) : 0u;
+                m.w0_l = lane < gsz ? __ldg(bitrow + page_word(L, m.pg0)) : 0u;
+                m.w1_l = lane < gsz ? __ldg(bitrow + page_word(L, m.pg1)) : 0u;
                 return true;
             }
             return false;
@@ -653,23 +680,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_parity = (n & 1u) ^ 1u;
             const int b = cur.b, h = cur.h, u0 = cur.u0, nU = has_cur ? cur.nU : 0;
             for (int j0 = 0; j0 < nU && !stop; j0 += 32) {
-                int phys = 0;
-                if (j0 + lane < nU) {
-                    const int pg = L.union_pages[u0 + j0 + lane];
-                    phys = L.page_table[static_cast<size_t>(b) * L.max_pages + pg];
-                    if (phys < 0 || phys >= L.n_phys) {
-                        set_status(L.status, PW_ERR_INVALID_ARG);
-                        phys = 0;
-                    }
-                }
+                const int phys = j0 + lane < nU ? phys_page(L, b, L.union_pages[u0 + j0 + lane]) : 0;
                 const int cnt = min(32, nU - j0); // j0 is even: a step never straddles chunks
                 for (int jj = 0; jj < cnt && !stop; jj += 2, ++stp) {
                     const int np = min(2, cnt - jj);
                     const int32_t row0 = (__shfl_sync(kFull, phys, jj) * L.Hkv + h) * 64;
                     const int32_t row1 = (__shfl_sync(kFull, phys, min(jj + 1, 31)) * L.Hkv + h) * 64;
                     // K: both pages of the step into one stage pair, on one barrier
+                    // the pair is free once S of step stp - 2 has completed
                     const uint32_t kp = stp % kNKP;
-                    if (!lwait(&sm.kst_empty[kp], ((stp / kNKP) & 1u) ^ 1u)) {
+                    if (!lwait(&sm.s_done[kp], ((stp / kNKP) & 1u) ^ 1u)) {
                         stop = true;
                         break;
                     }
@@ -716,41 +736,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             gi_next = nxt.gi + gstep;
         }
     } else if (warp == kWarpMma) {
-        // ---------------- MMA issue: the warp runs in lockstep, one elected lane issues ----------------
-        // Every lane polls the mbarriers and a vote makes each decision warp-uniform; operands
-        // are computed by the converged warp (uniform registers), the elected lane (always
-        // lane 0) issues the MMAs and their commits.  Per step n: S_n for the step's one or two
-        // pages (N = 64 or 128), then the products of the pages of step n - 1.
+        // ---------------- MMA issue ----------------
+        // The whole warp runs the loop in lockstep: every lane polls the mbarriers and a vote
+        // makes each decision warp-uniform; operands are computed by the converged warp and the
+        // elected lane (always lane 0) issues the tensor-core instructions and their commits.
+        // Per step n: S_n for the step's one or two pages (N = 64 or 128), then the products of
+        // step n - 1.  A step has four waits (K pair, S/P buffer free, P, V tiles) and two
+        // commits (S done, products done).
         auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             const bool ok = wait_bar(bar, parity, &sm.abort_flag); // every lane polls
             return __all_sync(kFull, ok);
         };
         const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
         const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // V, MN-major (dims contiguous)
-        uint32_t it = 0, stp = 0, nact = 0;
+        uint32_t stp = 0, nact = 0;
         bool have_prev = false, ok = true;
         // the step whose products are still to issue, kept in scalars
-        uint32_t pv_it0 = 0, pv_stp = 0, pv_np = 0, pv_nact = 0;
+        uint32_t pv_stp = 0, pv_np = 0, pv_nact = 0;
         bool pv_first = false, pv_last = false;
         auto issue_pv = [&]() -> bool {
-            const uint32_t ob = pv_nact & 1u;
-            if (!wwait(&sm.p_full[pv_stp & 1u], (pv_stp >> 1) & 1u))
+            const uint32_t ob = pv_nact & 1u, sb = pv_stp & 1u;
+            if (!wwait(&sm.p_full[sb], (pv_stp >> 1) & 1u) || !wwait(&sm.v_full[sb], (pv_stp >> 1) & 1u) ||
+                (pv_first && !wwait(&sm.o_free[ob], ((pv_nact >> 1) & 1u) ^ 1u)))
                 return false;
-            // O (M = 64 rows, N = 128 dims) += P_hi V + P_lo V, P read from TMEM where the
-            // softmax wrote it (the step's S buffer), V (K = keys, N = dims) from its MN-major
-            // f16 tile.
+            tc_fence_after();
+            // O += P V, P read from TMEM where the softmax wrote it (the step's S buffer), V
+            // (K = keys, N = dims) from its MN-major f16 tile.
             constexpr uint32_t idesc = idesc_f16_f32(64, 128, false, true);
             const uint32_t d = tmem + kColO + 128 * ob;
-            const uint32_t pa = tmem + kColS * (pv_stp & 1u);
-            for (uint32_t k = 0; k < pv_np; ++k) {
-                const uint32_t page = pv_it0 + k, vs = page % kNV;
-                const bool first = pv_first && k == 0;
-                if (!wwait(&sm.v_full[vs], (page / kNV) & 1u) ||
-                    (first && !wwait(&sm.o_free[ob], ((pv_nact >> 1) & 1u) ^ 1u)))
-                    return false;
-                tc_fence_after();
-                const uint64_t bd = desc_add(dmn, smem_u32(&sm.v[vs][0][0]));
-                if (elect_one()) {
+            const uint32_t pa = tmem + kColS * sb;
+            const uint64_t bd0 = desc_add(dmn, smem_u32(&sm.v[sb][0][0][0]));
+            if (elect_one()) {
+                for (uint32_t k = 0; k < pv_np; ++k) {
+                    const uint64_t bd = bd0 + ((k * sizeof(sm.v[0][0])) >> 4); // page k's tile
+                    const bool first = pv_first && k == 0;
                     // keys 16 kk .. 16 kk + 15: P_hi in columns 16 kk .. 16 kk + 7 of the page,
                     // P_lo in the next 8
 #pragma unroll
@@ -759,15 +778,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_f16_ts(d, a, bd + 128u * kk, idesc, (first && kk == 0) ? 0u : 1u);
                         mma_f16_ts(d, a + 8, bd + 128u * kk, idesc, 1u);
                     }
-                    mma_commit(&sm.v_empty[vs]);
-                    if (k + 1 == pv_np) {
-                        mma_commit(&sm.pvs_done[pv_stp & 1u]);
-                        if (pv_last)
-                            mma_commit(&sm.o_full[ob]);
-                    }
                 }
-                __syncwarp();
+                mma_commit(&sm.pvs_done[sb]);
+                if (pv_last)
+                    mma_commit(&sm.o_full[ob]);
             }
+            __syncwarp();
             return true;
         };
         for (;;) {
@@ -791,17 +807,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const uint32_t np = static_cast<uint32_t>(min(2, nU - s0));
-                const uint32_t kp = stp % kNKP, sb = stp & 1u;
+                const uint32_t sb = stp & 1u; // S/P buffer and K stage pair of the step
                 // S buffer sb holds the P of step stp - 2 (written by the softmax after it read S
-                // there): S may overwrite it once the products of that step have read it.  Their
-                // phase is one ahead of the one waited for two steps ago.
-                if (!wwait(&sm.kst_full[kp], (stp / kNKP) & 1u) ||
+                // there): S may overwrite it once the products of that step have read it.
+                if (!wwait(&sm.kst_full[sb], (stp >> 1) & 1u) ||
                     (stp >= 2 && !wwait(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[kp][0]));
+                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[sb][0]));
                 const uint32_t ds = tmem + kColS * sb;
                 const uint32_t idesc_s = idesc_e4m3_f32(64, static_cast<int>(64 * np));
                 if (elect_one()) {
@@ -813,7 +828,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, idesc_s, 1u);
                     mma_commit(&sm.s_done[sb]);
-                    mma_commit(&sm.kst_empty[kp]);
                     if (s0 + static_cast<int>(np) == nU)
                         mma_commit(&sm.q_empty[qb]);
                 }
@@ -822,14 +836,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                pv_it0 = it;
                 pv_stp = stp;
                 pv_np = np;
                 pv_nact = nact;
                 pv_first = s0 == 0;
                 pv_last = s0 + static_cast<int>(np) == nU;
                 have_prev = true;
-                it += np;
             }
             if (!ok)
                 break;
@@ -838,10 +850,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && have_prev)
             (void)issue_pv();
     } else if (warp < kWarpSm0) {
-        // ---------------- decode: E4M3 -> f16 V tiles ----------------
-        // One thread (tid 0) waits on each mbarrier; the others learn the outcome at named
-        // barrier kBarDecode.
-        uint32_t it = 0, nact = 0;
+        // ---------------- decode: E4M3 -> f16 V tiles, one step (one or two pages) at a time ----
+        // One thread (tid 0) waits on the mbarriers; the others learn the outcome at named barrier
+        // kBarDecode.  The tiles of step n go to step slot n % 2, free again once the products of
+        // step n - 2 are complete.
+        uint32_t it = 0, stp = 0, nact = 0;
         bool ok = true;
         for (;;) {
             const uint32_t jb = nact % kNJ;
@@ -854,23 +867,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             warp_arrive(&sm.job_empty[jb], lane);
             if (nU < 0)
                 break;
-            for (int j = 0; j < nU; ++j, ++it) {
-                const uint32_t st = it % kNSV, vs = it % kNV;
+            for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
+                const int np = min(2, nU - s0);
+                const uint32_t sb = stp & 1u, st0 = it % kNSV, st1 = (it + 1) % kNSV;
                 bool got = true;
                 if (tid == 0)
-                    got = wait_bar_c(&sm.vst_full[st], (it / kNSV) & 1u, &sm.abort_flag) &&
-                          wait_bar_c(&sm.v_empty[vs], ((it / kNV) & 1u) ^ 1u, &sm.abort_flag);
+                    got = (stp < 2 || wait_bar_c(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u, &sm.abort_flag)) &&
+                          wait_bar_c(&sm.vst_full[st0], (it / kNSV) & 1u, &sm.abort_flag) &&
+                          (np < 2 || wait_bar_c(&sm.vst_full[st1], ((it + 1) / kNSV) & 1u, &sm.abort_flag));
                 if (bar_or(kBarDecode, kDecThreads, !got)) {
                     ok = false;
                     break;
                 }
-                decode_page_f16<kDecThreads>(sm.stage_v[st], sm.v[vs], tid);
+#pragma unroll 1
+                for (int k = 0; k < np; ++k)
+                    decode_page_f16<kDecThreads>(sm.stage_v[k == 0 ? st0 : st1], sm.v[sb][k], tid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&sm.v_full[vs]);
-                    mbar_arrive(&sm.vst_empty[st]);
+                    mbar_arrive(&sm.v_full[sb]);
+                    mbar_arrive(&sm.vst_empty[st0]);
+                    if (np == 2)
+                        mbar_arrive(&sm.vst_empty[st1]);
                 }
+                it += np;
             }
             if (!ok)
                 break;
@@ -890,15 +910,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hw = sw >> 2;             // key half of each page read by this warp
         const int row = 16 * qd + (lane & 15);
         const int qq = 2 * hw + (lane >> 4); // 16-key quarter of each page owned by this thread
-        const float crow = L.sm_scale * L.k_scale * kLog2e;
-        const float acrow = fabsf(crow);
+        // |log2-domain factor|: when the factor is negative, the Q tile is negated instead
+        const float acrow = fabsf(L.sm_scale * L.k_scale * kLog2e);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        uint32_t it = 0, stp = 0, nact = 0, it_prev0 = 0;
-        // Products known complete: pages [0, pv_done).  Seeing S of step n proves the products
-        // of step n - 2 complete (they were issued before it); the slow path waits for the rest
-        // when it rescales.  Only the leader waits (every thread advances pv_done alike); the
-        // collective vote that follows passes the outcome on.
-        uint32_t pv_done = 0;
+        uint32_t stp = 0, nact = 0;
         auto allowed = [&](int pg, uint32_t word, int pos, int own) -> int { // keys of page pg in my quarter
             int n_allow = 0;
             if ((word >> (pg & 31)) & 1u)
@@ -930,7 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t *bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
             // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain factor
             const float inv = exp2i(-J.qexp[row]);
-            const float crow_r = crow * inv, acrow_r = acrow * inv;
+            const float c_r = acrow * inv;
             // Union page ids and my membership words, software-pipelined so that no step waits
             // on a global load: at the top of each step the words of the next step's pages and
             // the ids of the pages two steps ahead are requested; at its end, when they have
@@ -948,77 +963,72 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const int np = min(2, nU - s0);
                 if (s0 + 2 < nU && valid)
-                    wn0 = __ldg(bitrow + (pn0 >> 5));
+                    wn0 = __ldg(bitrow + page_word(L, pn0));
                 if (s0 + 3 < nU && valid)
-                    wn1 = __ldg(bitrow + (pn1 >> 5));
+                    wn1 = __ldg(bitrow + page_word(L, pn1));
                 if (s0 + 4 < nU)
                     pnn0 = L.union_pages[u0 + s0 + 4];
                 if (s0 + 5 < nU)
                     pnn1 = L.union_pages[u0 + s0 + 5];
                 const uint32_t sb = stp & 1u;
-                const uint32_t it0 = it;
                 // Every warp waits for S itself (all lanes poll, the warp decides by vote), so the
                 // warps are not lined up at a barrier here.  Every abort decision of this role is
                 // still collective (a thread that left alone would strand the others at the named
                 // barrier or in a warp-wide TMEM load): a warp whose wait gave up carries that to
                 // the vote below.
+                // The scores of both pages of the step arrive in one round trip and stay in
+                // registers for the max and for P.  For a one-page step the second page's
+                // columns hold stale values; they are all masked.
                 const bool s_ok = __all_sync(kFull, wait_bar(&sm.s_done[sb], (stp >> 1) & 1u, &sm.abort_flag));
-                if (pv_done < it_prev0)
-                    pv_done = it_prev0;
-                // S of the step is read twice (for the max, then for P), one page at a time, so
-                // that only sixteen scores are live in registers.
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_base + kColS * sb + 32 * hw;
+                uint32_t sa[16], sc[16];
+                tmem_ld_16x32bx2_x16(s_addr, sa);
+                tmem_ld_16x32bx2_x16(s_addr + 64, sc);
                 const int nqA = allowed(pgA, wA, pos, own);
                 const int nqB = np == 2 ? allowed(pgB, wB, pos, own) : 0;
-                const bool flip = crow < 0.f;
-                float lm;
-                {
-                    uint32_t sv[16];
-                    tmem_ld_16x32bx2_x16(s_addr, sv);
-                    tmem_ld_wait16(sv);
-                    lm = quarter_max(sv, nqA, flip);
-                    if (np == 2) {
-                        tmem_ld_16x32bx2_x16(s_addr + 64, sv);
-                        tmem_ld_wait16(sv);
-                        lm = fmaxf(lm, quarter_max(sv, nqB, flip));
-                    }
-                }
+                tmem_ld_wait2x16(sa, sc);
+                float lm = fmaxf(page_max(sa, nqA), page_max(sc, nqB));
                 const bool any = nqA > 0 || nqB > 0;
                 if (any)
-                    lm *= acrow_r;
+                    lm *= c_r;
                 if (softmax_bar_or(!s_ok || (any && lm > m_used + kRescaleLog2))) {
                     if (softmax_bar_or(!s_ok)) {
                         ok = false;
                         break;
                     }
                     const SlowOut so = softmax_slow_path(sm, row, qq, hw, any, lm, m_used, l_part, s0 == 0,
-                                                         it0 - 1, pv_done, sleader, o_addr);
+                                                         stp, sleader, o_addr);
                     m_used = so.m_used;
                     l_part = so.l_part;
-                    pv_done = so.pv_done;
                     if (!so.ok) {
                         ok = false;
                         break;
                     }
+                    // The scores again (still in TMEM): keeping them in registers across the
+                    // out-of-line call would spill them.
+                    tmem_ld_16x32bx2_x16(s_addr, sa);
+                    tmem_ld_16x32bx2_x16(s_addr + 64, sc);
+                    tmem_ld_wait2x16(sa, sc);
                 }
                 const float negm = m_used == -INFINITY ? 0.f : -m_used;
-                // P of each page goes back over that page's S columns (each thread over the 16 it
-                // read), where the products read it as their A operand.  The products of step
-                // stp - 2 read the same columns as P before S of this step overwrote them (the
-                // tensor pipe keeps issue order).
+                // P of each page goes back over that page's S columns, where the products read it
+                // as their A operand; the products of step stp - 2, which read these columns as P,
+                // completed before S of this step was issued.
+                // One call site for both pages (page 1's scores move into sa after page 0).
+#pragma unroll 1
                 for (int k = 0; k < np; ++k) {
-                    uint32_t sv[16];
-                    tc_fence_after();
-                    tmem_ld_16x32bx2_x16(s_addr + 64 * k, sv);
-                    tmem_ld_wait16(sv);
-                    l_part += emit_p(sv, k == 0 ? nqA : nqB, crow_r, negm, s_addr + 64 * k);
+                    uint32_t hi[8], lo[8];
+                    l_part += p_page(sa, k == 0 ? nqA : nqB, c_r, negm, hi, lo);
+                    store_p(hi, lo, s_addr + 64 * k);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        sa[e] = sc[e];
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 warp_arrive(&sm.p_full[sb], lane);
-                it_prev0 = it0;
-                it += np;
+
                 pgA = pn0;
                 pgB = pn1;
                 wA = wn0;
@@ -1053,6 +1063,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int et = tid - kWarpEpi0 * 32; // 0..127
         const bool eleader = et == 0;
         const uint32_t lane_base = static_cast<uint32_t>(32 * eq) << 16;
+        // The softmax works with |log2-domain factor|; a negative factor's sign goes into Q.
+        const float qsign = L.sm_scale * L.k_scale < 0.f ? -1.f : 1.f;
         // Q tile of group m: scaled, split into two E4M3 parts, written to buffer m % 2.
         // Returns false when a wait gave up; nU_out < 0 marks the end.
         auto prep_q = [&](uint32_t m, int &nU_out) -> bool {
@@ -1089,7 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     e = max(e, __shfl_xor_sync(kFull, e, o));
                 const int sexp = q_scale_exp(e);
                 uint2 q1, q2;
-                split_q8(val, exp2i(sexp), q1, q2);
+                split_q8(val, qsign * exp2i(sexp), q1, q2);
                 const uint32_t off = swz(row, c >> 1) + 8u * (c & 1);
                 *reinterpret_cast<uint2 *>(sm.q[qb][0] + off) = q1;
                 *reinterpret_cast<uint2 *>(sm.q[qb][1] + off) = q2;

@@ -11,7 +11,6 @@
 // device, so every GPU that loads the library holds it until the process exits.
 #include <cstddef>
 #include <cstdint>
-#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -25,28 +24,18 @@ constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(PW_NOALLOC_SCRATCH_B
 // device address must be fetched with cudaGetSymbolAddress (below), never taken directly.
 static __device__ __align__(256) unsigned char g_group_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Device address of g_group_scratch on the current device, looked up once per device.
+// Device address of g_group_scratch on the current device.  It is looked up on every call:
+// the address belongs to the module instance the runtime holds for the device, and a device
+// reset replaces that instance, so a cached address could outlive it.  The first lookup on a
+// device also loads the module there (with lazy loading), which is why the first call on a
+// device should come before any stream capture.
 cudaError_t scratch_on_current_device(void **out)
 {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_group_scratch);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_group_scratch);
-        if (e != cudaSuccess)
-            return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

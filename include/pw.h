@@ -17,7 +17,9 @@
  * Conventions shared by every entry point
  *   - Pointers are DEVICE pointers unless the parameter name ends in _host.
  *   - The caller owns and allocates every buffer (pw_groups_size reports the sizes); the
- *     library allocates no memory, keeps no global state and never synchronises the stream.
+ *     library allocates no memory and never synchronises the stream.  Its one piece of global
+ *     state is the fixed scratch array of pw_group_noalloc (below), which the CUDA runtime
+ *     places on every device that loads the library.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
  *   - The return value reports errors found on the host (arguments, launch failures).
  *     Errors that depend on the data (a selected page outside the query's causal prefix, a
@@ -152,9 +154,10 @@ pw_status pw_attn(const void *Q, const void *K_pages, const void *V_pages,
  * cudaMalloc, no cudaFree, no allocating library routine).
  *   - Shapes whose workspace (pw_groups_size) exceeds PW_NOALLOC_SCRATCH_BYTES are rejected
  *     with PW_ERR_CAPACITY before any device work; use pw_group with your own workspace then.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current) and caches it; make that first call before any stream capture.
- *     The stream must belong to the current device.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress), so the address stays valid across a device reset.  The first call
+ *     on a device also loads the library's device code there; make that first call before any
+ *     stream capture.  The stream must belong to the current device.
  *   - All calls on a device share the one array, which keeps the last call's contents.  Nothing
  *     in it needs clearing between calls, but calls that overlap on the GPU (different streams,
  *     no ordering between them) race on it and must not be issued.

@@ -54,17 +54,38 @@ def compare_rows(got_bits: np.ndarray, ref_f64: np.ndarray, what: str = ""):
     return max_abs, rel
 
 
-def sample_rows(wl: synth.Workload, groups: dict, n_random: int, seed: int = 0):
-    """(t, hq) rows: every row of the first, a middle and the last group of each kv head
-    (first/last sequence) plus n_random uniformly drawn rows."""
+def sample_rows(wl: synth.Workload, groups: dict, n_random: int, seed: int = 0,
+                n_ctas: int = 148, n_largest: int = 64):
+    """(t, hq) rows to compare at full size, chosen so that every group and every place where a
+    pipelined kernel changes state is covered:
+      - one row (random member, random head) of every group, so every group's union, page
+        steps and odd page counts are exercised;
+      - every row of the n_largest groups with the longest unions;
+      - every row of each persistent CTA's first and last group (the kernel walks the groups
+        gi, gi + n_ctas, ...), where its pipelines fill and drain;
+      - every row of the first, a middle and the last group;
+      - n_random uniformly drawn rows."""
     rng = np.random.default_rng(seed)
     G = wl.G
-    rows = set()
     n = groups["n_groups"]
-    picks = [0, n // 2, n - 1] if n > 0 else []
-    for gi in picks:
-        h = int(groups["gmeta"][gi, 1])
-        for t in groups["qids"][gi, : groups["gsize"][gi]]:
+    gsize = np.asarray(groups["gsize"][:n])
+    qids = np.asarray(groups["qids"][:n])
+    heads = np.asarray(groups["gmeta"][:n, 1])
+    usize = np.diff(np.asarray(groups["union_off"][: n + 1]))
+    rows = set()
+    if n > 0:
+        mem = (rng.random(n) * gsize).astype(np.int64)
+        hqs = heads * G + rng.integers(0, G, n)
+        for t, hq in zip(qids[np.arange(n), mem], hqs):
+            rows.add((int(t), int(hq)))
+    full = set([0, n // 2, n - 1] if n > 0 else [])
+    full.update(int(i) for i in np.argsort(-usize, kind="stable")[:n_largest])
+    c = min(n_ctas, n)
+    full.update(range(c))
+    full.update(range(max(n - c, 0), n))
+    for gi in full:
+        h = int(heads[gi])
+        for t in qids[gi, : gsize[gi]]:
             for j in range(G):
                 rows.add((int(t), h * G + j))
     for t, hq in zip(rng.integers(0, wl.T, n_random), rng.integers(0, wl.Hq, n_random)):

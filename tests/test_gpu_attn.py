@@ -1,8 +1,10 @@
 """pw_attn on the GPU against the oracle, element by element.
 
 Small cases compare every output row; the benchmark workloads at full size compare every row
-(workloads 1-2) or a sample of rows the oracle computes one by one (workloads 3-5), always in
-the same launch configuration the benchmark times (pw_group then pw_attn on one stream).
+(workloads 1-2) or, on workloads 3-5, rows the oracle computes one by one: one row of every
+group plus every row of the longest unions and of each persistent CTA's first and last group
+(parity.sample_rows), always in the same launch configuration the benchmark times (pw_group
+then pw_attn on one stream).
 """
 import numpy as np
 import pytest
@@ -114,10 +116,13 @@ def test_attn_full_workload_sampled_rows(cfg, W, g):
     got, gr = _run(inp, W, g)
     gh = gr.to_host()
     parity.assert_groups_equal(gh, parity.oracle_groups(wl, W, g))
-    rt, rh = parity.sample_rows(wl, gh, n_random=3000, seed=cfg)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    rt, rh = parity.sample_rows(wl, gh, n_random=3000, seed=cfg, n_ctas=n_sm)
     ref = oracle.attn_rows(inp, rt, rh)
     got = got.reshape(wl.T, wl.Hq, 128)[rt, rh]
-    parity.compare_rows(got, ref, f"{wl.name} W={W} g={g}")
+    max_abs, rel = parity.compare_rows(got, ref, f"{wl.name} W={W} g={g}")
+    print(f"{wl.name} W={W} g={g}: {len(rt)} rows of {wl.T * wl.Hq}, every group covered, "
+          f"max_abs {max_abs:.3e}, rel_l2 {rel:.3e}")
 
 
 @pytest.mark.parametrize("code", [0x01, 0x03, 0x07, 0x87, 0x08])
@@ -170,3 +175,52 @@ def test_q_rows_with_wide_dynamic_range():
     inp["Q"] = q.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     got, _ = _run(inp, 32, 8)
     parity.compare_rows(got.reshape(-1, 128), oracle.attn_all(inp).reshape(-1, 128), "wide Q rows")
+
+
+def _attn_raw(d, groups, max_pages, page_table, status):
+    """pw_attn straight through the C ABI (no binding-side checks), on the current stream."""
+    import ctypes as C
+    from dynamic_sparse_attention_pw_b200 import _lib
+    L = _lib.load()
+    Q = d["Q"]
+    T, Hq, _ = Q.shape
+    O = torch.zeros_like(Q)
+    st = groups.struct()
+    p = lambda t: C.c_void_p(t.data_ptr())
+    rc = L.pw_attn(p(Q), p(d["K_pages"]), p(d["V_pages"]), p(page_table), max_pages,
+                   d["K_pages"].shape[0], p(d["cu_seqlens"]), d["cu_seqlens"].numel() - 1, T, Hq,
+                   d["K_pages"].shape[1], 1.0, 1.0, float(d["sm_scale"]), C.byref(st), p(O),
+                   p(status), C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    return rc, int(status.item())
+
+
+def test_page_table_narrower_than_a_sequence_is_reported():
+    # The caller passes a page table with one column fewer than the sequence has pages: the
+    # kernel must not index past the row (the last page's id equals the row's width); it
+    # records PW_ERR_INVALID_ARG in the device status.  Every access stays inside the buffers.
+    wl = _small(16, [256], 4, 1, 4)
+    d = api.device_inputs(parity.inputs(wl))
+    status = api.new_status()
+    groups = api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], 32, 8, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    pt = d["page_table"]
+    assert pt.shape == (1, 4)
+    rc, code = _attn_raw(d, groups, pt.shape[1] - 1, pt, status)
+    assert rc == 0 and code == 1, (rc, code)        # PW_ERR_INVALID_ARG
+
+
+def test_page_table_entry_outside_the_pool_is_reported():
+    # A page table entry outside [0, n_phys) records PW_ERR_INVALID_ARG; the kernel reads slot
+    # 0 in its place, so nothing outside the K and V pools is read.
+    wl = _small(17, [256, 130], 4, 1, 4, shuffled_pages=True)
+    d = api.device_inputs(parity.inputs(wl))
+    status = api.new_status()
+    groups = api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], 32, 8, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    pt = d["page_table"].clone()
+    pt[1, 1] = d["K_pages"].shape[0]                  # one past the pool
+    rc, code = _attn_raw(d, groups, pt.shape[1], pt, status)
+    assert rc == 0 and code == 1, (rc, code)
