@@ -173,8 +173,11 @@ __device__ __noinline__ bool wait_bar_lazy(uint64_t *bar, uint32_t parity, int32
     }
 }
 
-// Named barriers, one per role that has more than one warp (0 is __syncthreads).
-constexpr uint32_t kBarSoftmax = 1, kBarDecode = 2, kBarEpilogue = 3;
+// Named barriers (0 is __syncthreads): the epilogue role has one; the softmax
+// role has one per TMEM lane quadrant (kBarSoftmax0 + quadrant), shared by the two warps that
+// hold that quadrant's rows, so that the quadrants never wait for one another.
+constexpr uint32_t kBarEpilogue = 3, kBarSoftmax0 = 4;
+constexpr uint32_t kSmQuadThreads = 64;
 
 // Named barrier `id` over `n` threads, returning whether any of them passed `pred`.  Warps
 // blocked here issue nothing, so one thread of a role waits on an mbarrier and the others wait
@@ -192,14 +195,15 @@ __device__ __forceinline__ bool bar_or(uint32_t id, uint32_t n, bool pred)
     return r != 0;
 }
 
-__device__ __forceinline__ bool softmax_bar_or(bool pred)
+// The softmax barrier of quadrant qd (its two warps).
+__device__ __forceinline__ bool softmax_bar_or(uint32_t qd, bool pred)
 {
-    return bar_or(kBarSoftmax, kSmThreads, pred);
+    return bar_or(kBarSoftmax0 + qd, kSmQuadThreads, pred);
 }
 
-__device__ __forceinline__ void softmax_bar()
+__device__ __forceinline__ void softmax_bar(uint32_t qd)
 {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(kBarSoftmax0 + qd), "r"(kSmQuadThreads) : "memory");
 }
 
 // One thread of a role (`leader`) waits on the mbarrier; the role's `n` threads learn the
@@ -291,6 +295,44 @@ __device__ __forceinline__ void split_q8(const uint4 v, float scale, uint2 &q1, 
     q2 = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
 }
 
+// Packed fp32 pairs: two independent IEEE single-precision operations per instruction.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// (x0, x1) = (s0, s1) * c2 + m2, elementwise (c2, m2 packed pairs).
+__device__ __forceinline__ void fma2(float &x0, float &x1, uint32_t s0, uint32_t s1, uint64_t c2, uint64_t m2)
+{
+    asm("{\n\t.reg .b64 s2, x2;\n\t"
+        "mov.b64 s2, {%2, %3};\n\t"
+        "fma.rn.f32x2 x2, s2, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, x2;\n\t}"
+        : "=f"(x0), "=f"(x1)
+        : "r"(s0), "r"(s1), "l"(c2), "l"(m2));
+}
+
+// a + (p0, p1), elementwise.
+__device__ __forceinline__ uint64_t add2(uint64_t a, float p0, float p1)
+{
+    uint64_t r;
+    asm("{\n\t.reg .b64 p2;\n\t"
+        "mov.b64 p2, {%1, %2};\n\t"
+        "add.rn.f32x2 %0, %3, p2;\n\t}"
+        : "=l"(r)
+        : "f"(p0), "f"(p1), "l"(a));
+    return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Largest of this thread's 16 scores of a page over its allowed keys (the first nq), -inf when
 // none is allowed.  Each thread takes the case of its own nq: a page not selected by the row's
 // query (nq = 0) costs nothing, a fully allowed one needs no predicates.
@@ -299,16 +341,14 @@ __device__ __forceinline__ float page_max(const uint32_t (&sv)[16], int nq)
     if (nq == 0)
         return -INFINITY;
     if (nq == 16) {
-        float m0 = __uint_as_float(sv[0]), m1 = __uint_as_float(sv[1]);
-        float m2 = __uint_as_float(sv[2]), m3 = __uint_as_float(sv[3]);
-#pragma unroll
-        for (int e = 4; e < 16; e += 4) {
-            m0 = fmaxf(m0, __uint_as_float(sv[e]));
-            m1 = fmaxf(m1, __uint_as_float(sv[e + 1]));
-            m2 = fmaxf(m2, __uint_as_float(sv[e + 2]));
-            m3 = fmaxf(m3, __uint_as_float(sv[e + 3]));
-        }
-        return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        const float *v = reinterpret_cast<const float *>(sv);
+        float a = max3f(v[0], v[1], v[2]), b = max3f(v[3], v[4], v[5]);
+        a = max3f(a, v[6], v[7]);
+        b = max3f(b, v[8], v[9]);
+        a = max3f(a, v[10], v[11]);
+        b = max3f(b, v[12], v[13]);
+        a = max3f(a, v[14], v[15]);
+        return fmaxf(a, b);
     }
     float lm = -INFINITY;
 #pragma unroll
@@ -406,13 +446,17 @@ __device__ __forceinline__ float p_page(const uint32_t (&sv)[16], int nq, float 
 {
     float sum = 0.f;
     if (nq == 16) {
+        const uint64_t c2 = pack2(c, c), m2 = pack2(negm, negm);
+        uint64_t sum2 = 0; // (0.f, 0.f)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm));
-            const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm));
-            sum += p0 + p1;
+            float x0, x1;
+            fma2(x0, x1, sv[2 * e], sv[2 * e + 1], c2, m2);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            sum2 = add2(sum2, p0, p1);
             split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
+        sum = __uint_as_float(static_cast<uint32_t>(sum2)) + __uint_as_float(static_cast<uint32_t>(sum2 >> 32));
     } else if (nq == 0) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -451,10 +495,10 @@ struct SlowOut {
 
 __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, int hw, bool any, float lm,
                                                   float m_used, float l_part, bool first_step,
-                                                  uint32_t stp, bool sleader, uint32_t o_addr)
+                                                  uint32_t stp, bool sleader, uint32_t o_addr, uint32_t qd)
 {
     sm.qmax[row][qq] = any ? lm : -INFINITY;
-    softmax_bar();
+    softmax_bar(qd);
     const float M = fmaxf(fmaxf(sm.qmax[row][0], sm.qmax[row][1]), fmaxf(sm.qmax[row][2], sm.qmax[row][3]));
     float alpha = 1.f;
     bool rescale = false;
@@ -467,13 +511,13 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
         m_used = M;
     }
     // (at a group's first step no row has a max yet, so none rescales)
-    if (!first_step && softmax_bar_or(rescale)) {
+    if (!first_step && softmax_bar_or(qd, rescale)) {
         // pvs_done of step stp - 1 covers every product issued before it.  Its phase is
         // unambiguous: S of this step was issued after the products of step stp - 2 had
         // completed, and the products of step stp + 1 cannot have run yet.
         const bool ok = !sleader ||
                         wait_bar(&sm.pvs_done[(stp - 1) & 1u], ((stp - 1) >> 1) & 1u, &sm.abort_flag);
-        if (softmax_bar_or(!ok))
+        if (softmax_bar_or(qd, !ok))
             return SlowOut{m_used, l_part, false};
         // O[r, :] *= alpha[r]: the row sits in this warp's lanes, and its four threads take 32
         // head dimensions each (lanes 0-15 dims 64 hw .. 64 hw + 31, lanes 16-31 the next 32).
@@ -851,15 +895,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             (void)issue_pv();
     } else if (warp < kWarpSm0) {
         // ---------------- decode: E4M3 -> f16 V tiles, one step (one or two pages) at a time ----
-        // One thread (tid 0) waits on the mbarriers; the others learn the outcome at named barrier
-        // kBarDecode.  The tiles of step n go to step slot n % 2, free again once the products of
-        // step n - 2 are complete.
+        // Each warp waits on the mbarriers itself (every lane polls, a vote decides), so the four
+        // warps never wait for one another.  The tiles of step n go to step slot n % 2, free again
+        // once the products of step n - 2 are complete.
+        auto dwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(kFull, wait_bar_c(bar, parity, &sm.abort_flag));
+        };
         uint32_t it = 0, stp = 0, nact = 0;
         bool ok = true;
         for (;;) {
             const uint32_t jb = nact % kNJ;
-            if (!role_wait(&sm.job_full[jb], (nact / kNJ) & 1u, &sm.abort_flag, tid == 0, kBarDecode,
-                           kDecThreads)) {
+            if (!dwait(&sm.job_full[jb], (nact / kNJ) & 1u)) {
                 ok = false;
                 break;
             }
@@ -870,12 +916,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const int np = min(2, nU - s0);
                 const uint32_t sb = stp & 1u, st0 = it % kNSV, st1 = (it + 1) % kNSV;
-                bool got = true;
-                if (tid == 0)
-                    got = (stp < 2 || wait_bar_c(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u, &sm.abort_flag)) &&
-                          wait_bar_c(&sm.vst_full[st0], (it / kNSV) & 1u, &sm.abort_flag) &&
-                          (np < 2 || wait_bar_c(&sm.vst_full[st1], ((it + 1) / kNSV) & 1u, &sm.abort_flag));
-                if (bar_or(kBarDecode, kDecThreads, !got)) {
+                if (!((stp < 2 || dwait(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u)) &&
+                      dwait(&sm.vst_full[st0], (it / kNSV) & 1u) &&
+                      (np < 2 || dwait(&sm.vst_full[st1], ((it + 1) / kNSV) & 1u)))) {
                     ok = false;
                     break;
                 }
@@ -905,7 +948,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // row exceeds its m by more than 2^8 (one OR over all 256 threads decides), so the
         // common path needs no exchange.
         const int sw = warp - kWarpSm0;     // 0..7
-        const bool sleader = sw == 0 && lane == 0; // the role's one mbarrier waiter
+        const bool sleader = sw < 4 && lane == 0; // the quadrant's one mbarrier waiter
         const int qd = sw & 3;              // TMEM lane quadrant
         const int hw = sw >> 2;             // key half of each page read by this warp
         const int row = 16 * qd + (lane & 15);
@@ -930,7 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (got && sm.job[jb].nU >= 0)
                     got = wait_bar_c(&sm.q_full[nact & 1u], (nact >> 1) & 1u, &sm.abort_flag);
             }
-            if (softmax_bar_or(!got)) {
+            if (softmax_bar_or(qd, !got)) {
                 ok = false;
                 break;
             }
@@ -992,13 +1035,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool any = nqA > 0 || nqB > 0;
                 if (any)
                     lm *= c_r;
-                if (softmax_bar_or(!s_ok || (any && lm > m_used + kRescaleLog2))) {
-                    if (softmax_bar_or(!s_ok)) {
+                if (softmax_bar_or(qd, !s_ok || (any && lm > m_used + kRescaleLog2))) {
+                    if (softmax_bar_or(qd, !s_ok)) {
                         ok = false;
                         break;
                     }
                     const SlowOut so = softmax_slow_path(sm, row, qq, hw, any, lm, m_used, l_part, s0 == 0,
-                                                         stp, sleader, o_addr);
+                                                         stp, sleader, o_addr, qd);
                     m_used = so.m_used;
                     l_part = so.l_part;
                     if (!so.ok) {
@@ -1041,7 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Publish the row-sum partials of this group for the epilogue warps.  lsum[ob] was
             // last read by the epilogue of group nact - 2, which released it with o_free[ob].
             ok = !sleader || wait_bar_c(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
-            if (softmax_bar_or(!ok)) {
+            if (softmax_bar_or(qd, !ok)) {
                 ok = false;
                 break;
             }
