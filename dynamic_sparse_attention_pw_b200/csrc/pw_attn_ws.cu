@@ -25,20 +25,24 @@
 //                         words, first page ids), the next group's Q rows by TMA, and the union
 //                         pages: K through a tensor map with the 128-byte swizzle the MMA reads,
 //                         V by bulk copy
-//   warp 17      MMA      S of step n (FP8, N = 64 per page) issued ahead of O += P V for step
-//                         n - 1
-// Few warps on purpose: the MMA warp sits on the critical path, and every extra busy warp on
-// its scheduler delays its waits and issues.  Compact code on purpose too: five roles run
+//   warp 17      MMA (S)  S (FP8, N = 64 per page) of each step, up to three steps ahead of
+//                         the products
+//   warp 18      MMA (PV) O += P V of each step
+// Few warps on purpose: the MMA warps sit on the critical path, and every extra busy warp on
+// their schedulers delays their waits and issues.  Compact code on purpose too: five roles run
 // different code on each scheduler, and on most SMs the kernel slows down in proportion to its
 // code size, so cold paths stay out of line or rolled and each role's loop calls each of its
 // steps from one place.
-// TMEM holds two S buffers and two O buffers (M = 64 layout: row r at lane 32 (r / 16) + r % 16).
-// The P of a step replaces its S in place, as the A operand of the products (keys 2j and 2j + 1
-// of a 16-key block packed in column j: P_hi in a block's first 8 columns, P_lo in the next 8).
-// Hand-offs per step, all mbarriers: S done (also frees the step's K stage pair), P written, V
-// tiles decoded, products done (frees the S/P buffer for S two steps later and the V step slot
-// for the tiles two steps later).  O is double-buffered across groups.  Every wait is bounded
-// and, when it runs out, sets an abort flag that releases the other roles.
+// TMEM holds three S/P buffers and one O buffer (M = 64 layout: row r at lane
+// 32 (r / 16) + r % 16).  The P of a step replaces its S in place, as the A operand of the products
+// (keys 2j and 2j + 1 of a 16-key block packed in column j: P_hi in a block's first 8 columns,
+// P_lo in the next 8).  S and the products are issued by two warps, so that neither stream's
+// waits hold up the other: S runs up to three steps ahead, as far as the buffers allow.
+// Hand-offs per step, all mbarriers: S done (also frees the step's K stage pair), P written and V
+// tiles decoded (one barrier), products done (frees the S/P buffer for S three steps later and
+// the V step slot for the tiles two steps later).  The first products of a group wait until the
+// epilogue has read the previous group's O.  Every wait is bounded and, when it runs out, sets an
+// abort flag that releases the other roles.
 #include <cstdint>
 #include <cuda.h> // CUtensorMap and its enums (the encoder itself is fetched at run time)
 #include <cuda_bf16.h>
@@ -54,21 +58,23 @@ namespace {
 
 using namespace attn;
 
-constexpr int kNKP = 2;       // E4M3 K stage pairs (one S step each), paired with the S buffers
+constexpr int kNS = 3;        // S/P buffers in TMEM, one step each
+constexpr int kNKP = kNS;     // E4M3 K stage pairs (one S step each), paired with the S buffers
 constexpr int kNSV = 4;       // E4M3 V page stages
 constexpr int kNJ = 3;        // group records in flight
 constexpr int kDecThreads = 128;
 constexpr int kSmThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kWarpSm0 = kDecThreads / 32, kWarpEpi0 = kWarpSm0 + 8, kWarpLoad = kWarpEpi0 + 4,
-              kWarpMma = kWarpLoad + 1;
-constexpr int kThreads = 32 * (kWarpMma + 1);
+              kWarpMma = kWarpLoad + 1, kWarpPv = kWarpMma + 1;
+constexpr int kThreads = 32 * (kWarpPv + 1);
 static_assert(kWarpSm0 % 4 == 0, "softmax warp w must sit in TMEM lane quadrant w % 4");
 static_assert(kWarpEpi0 % 4 == 0, "epilogue warp e must sit in TMEM lane quadrant e");
-static_assert(kNKP == 2, "a K stage pair is freed by the S completion of its S buffer");
-constexpr uint32_t kTmemCols = 512; // S / P [0..1] at columns 0 / 128, O[0..1] at 256 / 384
+static_assert(kNKP == kNS, "a K stage pair is freed by the S completion of its S buffer");
+constexpr uint32_t kTmemCols = 512; // S / P [0..2] at columns 0 / 128 / 256, O at 384
 constexpr uint32_t kColS = 128;     // one S step: two pages of 64 keys
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kColO = kColS * kNS;
+static_assert(kColO + 128 <= kTmemCols, "S/P buffers and O must fit in TMEM");
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // One group as the load warp hands it to the other roles, so that none of them meets a chain
@@ -91,22 +97,24 @@ struct __align__(1024) WsSmem {
     uint8_t q_raw[64 * 256];           // bf16 Q rows of the next group, row r at 256 r
     GroupJob job[kNJ];
     float qmax[64][4];    // per-row partial maxima exchanged by the row's four threads
-    float lsum[2][64][4]; // [O buffer][row][quarter]: per-thread partial row sums of a group
+    float lsum[2][64][4]; // [group % 2][row][quarter]: per-thread partial row sums of a group
     uint64_t job_full[kNJ], job_empty[kNJ];
     uint64_t qraw_full, qraw_empty;
     uint64_t kst_full[kNKP];
     uint64_t vst_full[kNSV], vst_empty[kNSV];
-    uint64_t v_full[2];   // v_full[n % 2]: the f16 V tiles of step n decoded
-    // s_done[n % 2]: S of step n complete; this also frees S's K stage pair (pair n % 2)
-    uint64_t s_done[2];
-    // pvs_done[n % 2]: the products of step n complete; this frees S/P buffer n % 2 for S of
-    // step n + 2 and the V step slot n % 2 for the tiles of step n + 2
-    uint64_t pvs_done[2];
-    uint64_t p_full[2];                 // p_full[n % 2]: P of both pages of step n written
+    // s_done[n % 3]: S of step n complete; this also frees S's K stage pair (pair n % 3)
+    uint64_t s_done[kNS];
+    // pvs_done[n % 3]: the products of step n complete; this frees S/P buffer n % 3 for S of
+    // step n + 3 and the V step slot n % 2 for the tiles of step n + 2
+    uint64_t pvs_done[kNS];
+    // pv_ready[n % 3]: P of step n written (one arrival per softmax warp) and its f16 V tiles
+    // decoded (one per decode warp): everything the products of step n read.  Neither role can
+    // arrive for step n + 3 before the products of step n are complete.
+    uint64_t pv_ready[kNS];
     uint64_t q_full[2], q_empty[2];
-    uint64_t o_full[2]; // last product of the group in O buffer b complete
-    uint64_t l_full[2]; // row sums of that group published
-    uint64_t o_free[2]; // epilogue done with O buffer b (and lsum[b])
+    uint64_t o_full;    // the last product of a group complete (one phase per group)
+    uint64_t l_full[2]; // l_full[g % 2]: the row sums of group g published
+    uint64_t o_free[2]; // o_free[g % 2]: the epilogue has read O and lsum[g % 2] of group g
     uint64_t drain_bar;
     uint32_t k_issued, v_issued; // steps / pages whose K / V copies the load warp issued
     uint32_t q_issued;           // groups whose Q rows it copied
@@ -114,6 +122,9 @@ struct __align__(1024) WsSmem {
     int32_t abort_flag;
     int32_t early_exit;
 };
+
+// The layout plus the slack for aligning it to 1024 bytes must fit one CTA's shared memory.
+static_assert(sizeof(WsSmem) + 1024 <= 227 * 1024, "shared-memory layout too large");
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 {
@@ -333,29 +344,35 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
     return r;
 }
 
-// Largest of this thread's 16 scores of a page over its allowed keys (the first nq), -inf when
-// none is allowed.  Each thread takes the case of its own nq: a page not selected by the row's
-// query (nq = 0) costs nothing, a fully allowed one needs no predicates.
+// A partial page (the query's own page, keys up to its position): the scores of the keys from
+// the nq-th on become -inf, so that the max and P of every page with allowed keys take one
+// path without per-key predicates (the log2-domain factor is kept positive, so -inf stays -inf
+// and its P is 0).
+__device__ __forceinline__ void mask_tail(uint32_t (&sv)[16], int nq)
+{
+    if (nq > 0 && nq < 16) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (e >= nq)
+                sv[e] = 0xFF800000u; // -inf
+    }
+}
+
+// Largest of this thread's 16 scores of a page (tail masked), -inf when no key is allowed.
+// Each thread takes the case of its own nq: a page not selected by the row's query (nq = 0)
+// costs nothing.
 __device__ __forceinline__ float page_max(const uint32_t (&sv)[16], int nq)
 {
     if (nq == 0)
         return -INFINITY;
-    if (nq == 16) {
-        const float *v = reinterpret_cast<const float *>(sv);
-        float a = max3f(v[0], v[1], v[2]), b = max3f(v[3], v[4], v[5]);
-        a = max3f(a, v[6], v[7]);
-        b = max3f(b, v[8], v[9]);
-        a = max3f(a, v[10], v[11]);
-        b = max3f(b, v[12], v[13]);
-        a = max3f(a, v[14], v[15]);
-        return fmaxf(a, b);
-    }
-    float lm = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-        if (e < nq)
-            lm = fmaxf(lm, __uint_as_float(sv[e]));
-    return lm;
+    const float *v = reinterpret_cast<const float *>(sv);
+    float a = max3f(v[0], v[1], v[2]), b = max3f(v[3], v[4], v[5]);
+    a = max3f(a, v[6], v[7]);
+    b = max3f(b, v[8], v[9]);
+    a = max3f(a, v[10], v[11]);
+    b = max3f(b, v[12], v[13]);
+    a = max3f(a, v[14], v[15]);
+    return fmaxf(a, b);
 }
 
 // p -> (hi, lo) f16 halves of two packed words: hi = p rounded to f16, lo = p - hi (exact in
@@ -439,13 +456,14 @@ __device__ __forceinline__ void tmem_ld_wait2x16(uint32_t (&a)[16], uint32_t (&b
 }
 
 // P = 2^(s c + negm) of the 16 keys of one row that this thread read of one page (the first nq
-// allowed, the rest 0), split into f16 hi + lo parts (keys 2j, 2j + 1 in word j).  Returns the
-// keys' sum.  As in page_max, each thread takes the case of its own nq.
+// allowed, the tail masked to -inf, so their P is 0), split into f16 hi + lo parts (keys 2j,
+// 2j + 1 in word j).  Returns the keys' sum.  As in page_max, each thread takes the case of its
+// own nq.
 __device__ __forceinline__ float p_page(const uint32_t (&sv)[16], int nq, float c, float negm,
                                         uint32_t (&hi)[8], uint32_t (&lo)[8])
 {
     float sum = 0.f;
-    if (nq == 16) {
+    if (nq != 0) { // every key allowed, or the tail masked to -inf
         const uint64_t c2 = pack2(c, c), m2 = pack2(negm, negm);
         uint64_t sum2 = 0; // (0.f, 0.f)
 #pragma unroll
@@ -457,18 +475,10 @@ __device__ __forceinline__ float p_page(const uint32_t (&sv)[16], int nq, float 
             split_pair_f16_pos(p0, p1, hi[e], lo[e]);
         }
         sum = __uint_as_float(static_cast<uint32_t>(sum2)) + __uint_as_float(static_cast<uint32_t>(sum2 >> 32));
-    } else if (nq == 0) {
+    } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             hi[e] = lo[e] = 0u;
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float p0 = 2 * e < nq ? ex2(fmaf(__uint_as_float(sv[2 * e]), c, negm)) : 0.f;
-            const float p1 = 2 * e + 1 < nq ? ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, negm)) : 0.f;
-            sum += p0 + p1;
-            split_pair_f16_pos(p0, p1, hi[e], lo[e]);
-        }
     }
     return sum;
 }
@@ -513,10 +523,10 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
     // (at a group's first step no row has a max yet, so none rescales)
     if (!first_step && softmax_bar_or(qd, rescale)) {
         // pvs_done of step stp - 1 covers every product issued before it.  Its phase is
-        // unambiguous: S of this step was issued after the products of step stp - 2 had
-        // completed, and the products of step stp + 1 cannot have run yet.
+        // unambiguous: S of this step was issued after the products of step stp - 3 had
+        // completed, and the products of step stp + 2 cannot have run yet.
         const bool ok = !sleader ||
-                        wait_bar(&sm.pvs_done[(stp - 1) & 1u], ((stp - 1) >> 1) & 1u, &sm.abort_flag);
+                        wait_bar(&sm.pvs_done[(stp - 1) % kNS], ((stp - 1) / kNS) & 1u, &sm.abort_flag);
         if (softmax_bar_or(qd, !ok))
             return SlowOut{m_used, l_part, false};
         // O[r, :] *= alpha[r]: the row sits in this warp's lanes, and its four threads take 32
@@ -554,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Arrivals from the decode and softmax roles are one per warp (after __syncwarp).
         for (int s = 0; s < kNJ; ++s) {
             mbar_init(&sm.job_full[s], 1);
-            mbar_init(&sm.job_empty[s], kDecThreads / 32 + 1 + kSmThreads / 32 + kEpiThreads / 32);
+            mbar_init(&sm.job_empty[s], kDecThreads / 32 + 2 + kSmThreads / 32 + kEpiThreads / 32);
         }
         mbar_init(&sm.qraw_full, 1);
         mbar_init(&sm.qraw_empty, kEpiThreads / 32);
@@ -564,18 +574,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.vst_full[s], 1);
             mbar_init(&sm.vst_empty[s], kDecThreads / 32);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.v_full[s], kDecThreads / 32);
+        for (int s = 0; s < kNS; ++s) {
             mbar_init(&sm.s_done[s], 1);
             mbar_init(&sm.pvs_done[s], 1);
-            mbar_init(&sm.p_full[s], kSmThreads / 32);
+            mbar_init(&sm.pv_ready[s], kSmThreads / 32 + kDecThreads / 32);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.q_full[s], kEpiThreads / 32);
             mbar_init(&sm.q_empty[s], 1);
-            mbar_init(&sm.o_full[s], 1);
             mbar_init(&sm.l_full[s], kSmThreads / 32);
             mbar_init(&sm.o_free[s], kEpiThreads / 32);
         }
-        mbar_init(&sm.drain_bar, 1);
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.drain_bar, 2); // one commit from each MMA-issuing warp
         sm.abort_flag = 0;
         sm.k_issued = 0;
         sm.v_issued = 0;
@@ -731,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t row0 = (__shfl_sync(kFull, phys, jj) * L.Hkv + h) * 64;
                     const int32_t row1 = (__shfl_sync(kFull, phys, min(jj + 1, 31)) * L.Hkv + h) * 64;
                     // K: both pages of the step into one stage pair, on one barrier
-                    // the pair is free once S of step stp - 2 has completed
+                    // the pair is free once S of step stp - 3 has completed
                     const uint32_t kp = stp % kNKP;
                     if (!lwait(&sm.s_done[kp], ((stp / kNKP) & 1u) ^ 1u)) {
                         stop = true;
@@ -779,63 +790,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             has_cur = true;
             gi_next = nxt.gi + gstep;
         }
-    } else if (warp == kWarpMma) {
-        // ---------------- MMA issue ----------------
-        // The whole warp runs the loop in lockstep: every lane polls the mbarriers and a vote
-        // makes each decision warp-uniform; operands are computed by the converged warp and the
-        // elected lane (always lane 0) issues the tensor-core instructions and their commits.
-        // Per step n: S_n for the step's one or two pages (N = 64 or 128), then the products of
-        // step n - 1.  A step has four waits (K pair, S/P buffer free, P, V tiles) and two
-        // commits (S done, products done).
+    } else if (warp == kWarpMma || warp == kWarpPv) {
+        // ---------------- MMA issue: two warps ----------------
+        // Warp kWarpMma issues S of every step, as soon as its K pair has landed and the products
+        // of the step three before (which read its S/P buffer as P) are complete, so it runs up
+        // to three steps ahead; warp kWarpPv issues O += P V of every step once its P is written
+        // and its V tiles decoded.  Each warp runs its loop in lockstep: every lane polls the
+        // mbarriers and a vote makes each decision warp-uniform; the elected lane (always lane
+        // 0) issues the tensor-core instructions and the commits, which track that lane's MMAs.
         auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
             const bool ok = wait_bar(bar, parity, &sm.abort_flag); // every lane polls
             return __all_sync(kFull, ok);
         };
+        const bool is_s = warp == kWarpMma;
         const uint64_t dsw = sdesc_sw128(0u, 16, 1024);    // K-major, address added below
         const uint64_t dmn = sdesc_sw128(0u, 8192, 1024);  // V, MN-major (dims contiguous)
-        uint32_t stp = 0, nact = 0;
-        bool have_prev = false, ok = true;
-        // the step whose products are still to issue, kept in scalars
-        uint32_t pv_stp = 0, pv_np = 0, pv_nact = 0;
-        bool pv_first = false, pv_last = false;
-        auto issue_pv = [&]() -> bool {
-            const uint32_t ob = pv_nact & 1u, sb = pv_stp & 1u;
-            if (!wwait(&sm.p_full[sb], (pv_stp >> 1) & 1u) || !wwait(&sm.v_full[sb], (pv_stp >> 1) & 1u) ||
-                (pv_first && !wwait(&sm.o_free[ob], ((pv_nact >> 1) & 1u) ^ 1u)))
-                return false;
-            tc_fence_after();
-            // O += P V, P read from TMEM where the softmax wrote it (the step's S buffer), V
-            // (K = keys, N = dims) from its MN-major f16 tile.
-            constexpr uint32_t idesc = idesc_f16_f32(64, 128, false, true);
-            const uint32_t d = tmem + kColO + 128 * ob;
-            const uint32_t pa = tmem + kColS * sb;
-            const uint64_t bd0 = desc_add(dmn, smem_u32(&sm.v[sb][0][0][0]));
-            if (elect_one()) {
-                for (uint32_t k = 0; k < pv_np; ++k) {
-                    const uint64_t bd = bd0 + ((k * sizeof(sm.v[0][0])) >> 4); // page k's tile
-                    const bool first = pv_first && k == 0;
-                    // keys 16 kk .. 16 kk + 15: P_hi in columns 16 kk .. 16 kk + 7 of the page,
-                    // P_lo in the next 8
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t a = pa + 64 * k + 16 * kk;
-                        mma_f16_ts(d, a, bd + 128u * kk, idesc, (first && kk == 0) ? 0u : 1u);
-                        mma_f16_ts(d, a + 8, bd + 128u * kk, idesc, 1u);
-                    }
-                }
-                mma_commit(&sm.pvs_done[sb]);
-                if (pv_last)
-                    mma_commit(&sm.o_full[ob]);
-            }
-            __syncwarp();
-            return true;
-        };
-        for (;;) {
+        constexpr uint32_t idesc_pv = idesc_f16_f32(64, 128, false, true);
+        uint32_t stp = 0;
+        bool ok = true;
+        for (uint32_t nact = 0; ok; ++nact) {
             const uint32_t jb = nact % kNJ;
-            if (!wwait(&sm.job_full[jb], (nact / kNJ) & 1u)) {
-                ok = false;
+            if (!wwait(&sm.job_full[jb], (nact / kNJ) & 1u))
                 break;
-            }
             const int nU = sm.job[jb].nU;
             __syncwarp();
             if (lane == 0)
@@ -843,56 +819,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nU < 0)
                 break;
             const uint32_t qb = nact & 1u;
-            if (!wwait(&sm.q_full[qb], (nact >> 1) & 1u)) {
-                ok = false;
-                break;
+            uint64_t aq1 = 0, aq2 = 0;
+            if (is_s) {
+                if (!wwait(&sm.q_full[qb], (nact >> 1) & 1u))
+                    break;
+                aq1 = desc_add(dsw, smem_u32(sm.q[qb][0]));
+                aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
             }
-            const uint64_t aq1 = desc_add(dsw, smem_u32(sm.q[qb][0]));
-            const uint64_t aq2 = desc_add(dsw, smem_u32(sm.q[qb][1]));
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const uint32_t np = static_cast<uint32_t>(min(2, nU - s0));
-                const uint32_t sb = stp & 1u; // S/P buffer and K stage pair of the step
-                // S buffer sb holds the P of step stp - 2 (written by the softmax after it read S
-                // there): S may overwrite it once the products of that step have read it.
-                if (!wwait(&sm.kst_full[sb], (stp >> 1) & 1u) ||
-                    (stp >= 2 && !wwait(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[sb][0]));
-                const uint32_t ds = tmem + kColS * sb;
-                const uint32_t idesc_s = idesc_e4m3_f32(64, static_cast<int>(64 * np));
-                if (elect_one()) {
-                    // S' = q1 K^T + q2 K^T: four k-steps of 32 dims for each part
+                const bool last = s0 + static_cast<int>(np) == nU;
+                const uint32_t sb = stp % kNS; // S/P buffer (and K stage pair) of the step
+                if (is_s) {
+                    // S buffer sb holds the P of step stp - 3: S may overwrite it once the
+                    // products of that step have read it.
+                    if (!wwait(&sm.kst_full[sb], (stp / kNS) & 1u) ||
+                        (stp >= kNS && !wwait(&sm.pvs_done[sb], ((stp / kNS) & 1u) ^ 1u))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t bk = desc_add(dsw, smem_u32(sm.stage_k[sb][0]));
+                    const uint32_t ds = tmem + kColS * sb;
+                    const uint32_t idesc_s = idesc_e4m3_f32(64, static_cast<int>(64 * np));
+                    if (elect_one()) {
+                        // S' = q1 K^T + q2 K^T: four k-steps of 32 dims for each part
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f8_ss(ds, aq1 + 2u * kk, bk + 2u * kk, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f8_ss(ds, aq1 + 2u * kk, bk + 2u * kk, idesc_s, kk > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, idesc_s, 1u);
-                    mma_commit(&sm.s_done[sb]);
-                    if (s0 + static_cast<int>(np) == nU)
-                        mma_commit(&sm.q_empty[qb]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f8_ss(ds, aq2 + 2u * kk, bk + 2u * kk, idesc_s, 1u);
+                        mma_commit(&sm.s_done[sb]);
+                        if (last)
+                            mma_commit(&sm.q_empty[qb]);
+                    }
+                    __syncwarp();
+                } else {
+                    // P of the step in S/P buffer sb, its V tiles in step slot stp % 2; the first
+                    // products of group g overwrite O, so the epilogue must have read group
+                    // g - 1's.
+                    const uint32_t vsl = stp & 1u;
+                    if (!wwait(&sm.pv_ready[sb], (stp / kNS) & 1u) ||
+                        (s0 == 0 && nact > 0 && !wwait(&sm.o_free[(nact - 1) & 1u], ((nact - 1) >> 1) & 1u))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // O += P V, P read from TMEM where the softmax wrote it (the step's S buffer),
+                    // V (K = keys, N = dims) from its MN-major f16 tile.
+                    const uint32_t d = tmem + kColO;
+                    const uint32_t pa = tmem + kColS * sb;
+                    const uint64_t bd0 = desc_add(dmn, smem_u32(&sm.v[vsl][0][0][0]));
+                    if (elect_one()) {
+                        for (uint32_t k = 0; k < np; ++k) {
+                            const uint64_t bd = bd0 + ((k * sizeof(sm.v[0][0])) >> 4); // page k's tile
+                            const bool first = s0 == 0 && k == 0;
+                            // keys 16 kk .. 16 kk + 15: P_hi in columns 16 kk .. 16 kk + 7 of the
+                            // page, P_lo in the next 8
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t a = pa + 64 * k + 16 * kk;
+                                mma_f16_ts(d, a, bd + 128u * kk, idesc_pv, (first && kk == 0) ? 0u : 1u);
+                                mma_f16_ts(d, a + 8, bd + 128u * kk, idesc_pv, 1u);
+                            }
+                        }
+                        mma_commit(&sm.pvs_done[sb]);
+                        if (last)
+                            mma_commit(&sm.o_full);
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
-                if (have_prev && !issue_pv()) {
-                    ok = false;
-                    break;
-                }
-                pv_stp = stp;
-                pv_np = np;
-                pv_nact = nact;
-                pv_first = s0 == 0;
-                pv_last = s0 + static_cast<int>(np) == nU;
-                have_prev = true;
             }
-            if (!ok)
-                break;
-            ++nact;
         }
-        if (ok && have_prev)
-            (void)issue_pv();
     } else if (warp < kWarpSm0) {
         // ---------------- decode: E4M3 -> f16 V tiles, one step (one or two pages) at a time ----
         // Each warp waits on the mbarriers itself (every lane polls, a vote decides), so the four
@@ -915,8 +914,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const int np = min(2, nU - s0);
+                // V step slot sb was last read by the products of step stp - 2.  Their phase of
+                // pvs_done is unambiguous: this warp waited for those of step stp - 5 before
+                // decoding step stp - 3, and the products of step stp + 1 need tiles not yet made.
                 const uint32_t sb = stp & 1u, st0 = it % kNSV, st1 = (it + 1) % kNSV;
-                if (!((stp < 2 || dwait(&sm.pvs_done[sb], ((stp - 2) >> 1) & 1u)) &&
+                if (!((stp < 2 || dwait(&sm.pvs_done[(stp - 2) % kNS], ((stp - 2) / kNS) & 1u)) &&
                       dwait(&sm.vst_full[st0], (it / kNSV) & 1u) &&
                       (np < 2 || dwait(&sm.vst_full[st1], ((it + 1) / kNSV) & 1u)))) {
                     ok = false;
@@ -928,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&sm.v_full[sb]);
+                    mbar_arrive(&sm.pv_ready[stp % kNS]);
                     mbar_arrive(&sm.vst_empty[st0]);
                     if (np == 2)
                         mbar_arrive(&sm.vst_empty[st1]);
@@ -988,7 +990,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t *bitrow = L.bits + (static_cast<size_t>(tok) * L.Hkv + h) * L.words;
             // S arrives scaled by 2^s (the row's Q scale): fold 2^-s into the log2-domain factor
             const float inv = exp2i(-J.qexp[row]);
-            const float c_r = acrow * inv;
+            // (floored at a tiny positive value, so that a masked key's -inf score never meets a
+            // zero factor; a zero factor makes all allowed keys equal either way)
+            const float c_r = fmaxf(acrow * inv, 1e-30f);
             // Union page ids and my membership words, software-pipelined so that no step waits
             // on a global load: at the top of each step the words of the next step's pages and
             // the ids of the pages two steps ahead are requested; at its end, when they have
@@ -1000,8 +1004,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t wn0 = 0u, wn1 = 0u;      // next step (words requested at the top of this one)
             int pnn0 = pn0, pnn1 = pn1;       // two steps ahead (ids requested at the top of this one)
             warp_arrive(&sm.job_empty[jb], lane);
-            const uint32_t ob = nact & 1u;
-            const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
+            const uint32_t ob = nact & 1u; // lsum buffer of the group
+            const uint32_t o_addr = tmem + lane_base + kColO;
             float m_used = -INFINITY, l_part = 0.f;
             for (int s0 = 0; s0 < nU; s0 += 2, ++stp) {
                 const int np = min(2, nU - s0);
@@ -1013,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pnn0 = L.union_pages[u0 + s0 + 4];
                 if (s0 + 5 < nU)
                     pnn1 = L.union_pages[u0 + s0 + 5];
-                const uint32_t sb = stp & 1u;
+                const uint32_t sb = stp % kNS;
                 // Every warp waits for S itself (all lanes poll, the warp decides by vote), so the
                 // warps are not lined up at a barrier here.  Every abort decision of this role is
                 // still collective (a thread that left alone would strand the others at the named
@@ -1022,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // The scores of both pages of the step arrive in one round trip and stay in
                 // registers for the max and for P.  For a one-page step the second page's
                 // columns hold stale values; they are all masked.
-                const bool s_ok = __all_sync(kFull, wait_bar(&sm.s_done[sb], (stp >> 1) & 1u, &sm.abort_flag));
+                const bool s_ok = __all_sync(kFull, wait_bar(&sm.s_done[sb], (stp / kNS) & 1u, &sm.abort_flag));
                 tc_fence_after();
                 const uint32_t s_addr = tmem + lane_base + kColS * sb + 32 * hw;
                 uint32_t sa[16], sc[16];
@@ -1031,6 +1035,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nqA = allowed(pgA, wA, pos, own);
                 const int nqB = np == 2 ? allowed(pgB, wB, pos, own) : 0;
                 tmem_ld_wait2x16(sa, sc);
+                mask_tail(sa, nqA);
+                mask_tail(sc, nqB);
                 float lm = fmaxf(page_max(sa, nqA), page_max(sc, nqB));
                 const bool any = nqA > 0 || nqB > 0;
                 if (any)
@@ -1053,10 +1059,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_16x32bx2_x16(s_addr, sa);
                     tmem_ld_16x32bx2_x16(s_addr + 64, sc);
                     tmem_ld_wait2x16(sa, sc);
+                    mask_tail(sa, nqA);
+                    mask_tail(sc, nqB);
                 }
                 const float negm = m_used == -INFINITY ? 0.f : -m_used;
                 // P of each page goes back over that page's S columns, where the products read it
-                // as their A operand; the products of step stp - 2, which read these columns as P,
+                // as their A operand; the products of step stp - 3, which read these columns as P,
                 // completed before S of this step was issued.
                 // One call site for both pages (page 1's scores move into sa after page 0).
 #pragma unroll 1
@@ -1070,7 +1078,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_st_wait();
                 tc_fence_before();
-                warp_arrive(&sm.p_full[sb], lane);
+                warp_arrive(&sm.pv_ready[sb], lane);
 
                 pgA = pn0;
                 pgB = pn1;
@@ -1083,6 +1091,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             // Publish the row-sum partials of this group for the epilogue warps.  lsum[ob] was
             // last read by the epilogue of group nact - 2, which released it with o_free[ob].
+            // (The phase is unambiguous: S of this group's steps implies the products of group
+            // nact - 3, and so the epilogue's read of group nact - 4, are complete.)
             ok = !sleader || wait_bar_c(&sm.o_free[ob], ((nact >> 1) & 1u) ^ 1u, &sm.abort_flag);
             if (softmax_bar_or(qd, !ok)) {
                 ok = false;
@@ -1171,12 +1181,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // output of group n = m - 1
             const uint32_t n = m - 1;
-            const uint32_t jb = n % kNJ, ob = n & 1u;
+            const uint32_t jb = n % kNJ, ob = n & 1u; // lsum buffer of the group
             const GroupJob &J = sm.job[jb];
             const int h = J.h, R = J.R;
             bool got = true;
             if (eleader)
-                got = wait_bar_lazy(&sm.o_full[ob], (n >> 1) & 1u, &sm.abort_flag) &&
+                got = wait_bar_lazy(&sm.o_full, n & 1u, &sm.abort_flag) &&
                       wait_bar_lazy(&sm.l_full[ob], (n >> 1) & 1u, &sm.abort_flag);
             if (bar_or(kBarEpilogue, kEpiThreads, !got))
                 break;
@@ -1184,7 +1194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // along the columns.  Warp eq takes rows 16 eq .. 16 eq + 15; lanes 0-15 and 16-31
             // take 32 dimensions each per load, so each thread writes 64 contiguous bytes of a row.
             tc_fence_after();
-            const uint32_t o_addr = tmem + lane_base + kColO + 128 * ob;
+            const uint32_t o_addr = tmem + lane_base + kColO;
             const int r = 16 * eq + (lane & 15), half = lane >> 4;
             float inv = 0.f;
             uint16_t *orow = nullptr;
@@ -1240,7 +1250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (sm.q_issued > 0)
                 (void)mbar_wait(&sm.qraw_full, (sm.q_issued - 1) & 1u);
         }
-        if (warp == kWarpMma) {
+        if (warp == kWarpMma || warp == kWarpPv) { // each commit covers its own warp's MMAs
             if (elect_one()) {
                 mma_commit(&sm.drain_bar);
                 (void)mbar_wait(&sm.drain_bar, 0);
