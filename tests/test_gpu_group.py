@@ -36,6 +36,11 @@ SMALL = [
     (_small(6, [513], 2, 1, 9), 32, 1),
     (_small(7, [2048, 31], 4, 2, 40), 128, 32),
     (_small(8, [70000], 2, 1, 6), 128, 8),         # 1094 pages: two bitset words per lane
+    # more than 8 bitset words: windows renumbered to their own pages before the search
+    (_small(9, [20000, 3000], 4, 2, 24, "community", communities=8), 64, 8),
+    (_small(10, [40000], 2, 1, 16, "community", communities=16), 256, 4),
+    # uniform selections: later windows hold more than 256 distinct pages and are staged whole
+    (_small(11, [30000, 500], 4, 2, 40), 128, 8),
 ]
 
 
