@@ -439,10 +439,80 @@ def breakdown(wk, group_ms, attn_ms, step_ms, warm_ms, hbm, bf16):
 
 
 # The per-configuration runs of the measurement plan: the 64K workload swept over W, the 32K
-# workload grouped three ways (contiguous W = g, regrouped W = 128, one query per group), and the
-# remaining workloads at their own W.
+# workload grouped four ways (contiguous W = g, regrouped W = 128, one query per group, and
+# sixteen queries per group, whose 16 x 4 rows fill the 64-row tile that eight queries fill
+# only half of), and the remaining workloads at their own W.
 SWEEP = [(4, 32, 8), (4, 64, 8), (4, 256, 8), (3, 8, 8), (3, 128, 8), (3, 128, 1),
-         (1, 32, 8), (2, 64, 8), (5, 128, 8)]
+         (3, 128, 16), (1, 32, 8), (2, 64, 8), (5, 128, 8)]
+
+
+def launches_per_call(words, W):
+    """Kernels of one complete call: pw_group's bitset, greedy (plus the renumbering greedy for
+    windows whose staged rows would exceed 2112 words), offset and page kernels, then pw_attn."""
+    return 5 + (1 if words > 8 and words * (W + 1) > 2112 else 0)
+
+
+def run_overlap(dev, inp, W, steps, warmup=3):
+    """Grouping of call n + 1 on a second stream beside the attention of call n (two sets of
+    group buffers and status words), against the same calls one after the other.  Returns the
+    mean ms per call of each schedule; the 64K workload's inputs exceed L2, so no flush."""
+    import torch
+    from dynamic_sparse_attention_pw_b200 import api, synth
+    wl = synth.WORKLOADS[4].with_(W=W, g=8)
+    t = Timed(wl, W, 8, dev, inp=inp)
+    d = t.d
+    bufs = [(t.groups, t.status),
+            (api.Groups.allocate(wl.T, wl.Hkv, inp["cu_seqlens"], wl.kmax, W, 8, dev),
+             api.new_status(dev))]
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream(dev)
+
+    def group(i, stream):
+        g_, st = bufs[i % 2]
+        api.pw_group(d["sel_pages"], d["cu_seqlens"], d["cu_seqlens_host"], W, 8, groups=g_,
+                     status=st, stream=stream)
+
+    def attn(i, stream):
+        g_, st = bufs[i % 2]
+        api.pw_attn(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], d["cu_seqlens"], g_,
+                    d["k_scale"], d["v_scale"], d["sm_scale"], O=t.O, status=st, stream=stream)
+
+    n = warmup + steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    # one after the other, on one stream
+    seq = [ev() for _ in range(2)]
+    for i in range(n):
+        if i == warmup:
+            seq[0].record(main)
+        group(i, main)
+        attn(i, main)
+    seq[1].record(main)
+    torch.cuda.synchronize()
+    # overlapped: grouping i + 1 (side) waits only for attention i - 1, which read its buffers
+    gdone = [torch.cuda.Event() for _ in range(n + 1)]
+    adone = [torch.cuda.Event() for _ in range(n)]
+    ovl = [ev() for _ in range(2)]
+    side.wait_stream(main)
+    group(0, side)
+    gdone[0].record(side)
+    for i in range(n):
+        if i >= 1:
+            side.wait_event(adone[i - 1])
+        if i + 1 < n:
+            group(i + 1, side)
+            gdone[i + 1].record(side)
+        main.wait_event(gdone[i])
+        if i == warmup:
+            ovl[0].record(main)
+        attn(i, main)
+        adone[i].record(main)
+    ovl[1].record(main)
+    main.wait_stream(side)
+    torch.cuda.synchronize()
+    for _, st in bufs:
+        api.check_status(st, f"{wl.name} overlapped calls")
+    return {"workload": wl.name, "W": W, "g": 8, "steps": steps,
+            "sequential_ms_per_call": seq[0].elapsed_time(seq[1]) / steps,
+            "overlapped_ms_per_call": ovl[0].elapsed_time(ovl[1]) / steps}
 
 
 def run_sweep(args, dev, flush, clocks, hbm, bf16, head_inp):
@@ -562,9 +632,11 @@ def run_ours(args):
         return 0
 
     hbm, bf16, src = peaks()
-    sweep = None
+    sweep = overlap = None
     if not args.no_sweep and world == 1:
         sweep = run_sweep(args, dev, flush, clocks, hbm, bf16, head.inp)
+        if args.workload == 4:
+            overlap = [run_overlap(dev, head.inp, W, args.sweep_steps) for W in (128, 256)]
     clocks.__exit__(None, None, None)
 
     bd = breakdown(wk, group_ms, attn_ms, step_ms, warm_ms, hbm, bf16)
@@ -601,12 +673,14 @@ def run_ours(args):
         },
         "breakdown": bd,
         "clocks": clocks.summary(),
-        "gpu_launches": 5 * K,
+        "gpu_launches": launches_per_call(head.groups.words, args.W) * K,
     }
     if e2e is not None:
         line["e2e"] = e2e
     if sweep is not None:
         line["sweep"] = sweep
+    if overlap is not None:
+        line["grouping_overlap"] = overlap
     if not args.no_cpu_baseline and world == 1:
         rate, threads, desc, _, _ = oracle_sample(head.inp, wl, args.W, args.g, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s (useful)", "cores": threads,

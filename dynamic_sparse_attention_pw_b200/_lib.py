@@ -25,6 +25,7 @@ class PwGroups(C.Structure):
         ("union_off", C.c_void_p),
         ("union_pages", C.c_void_p),
         ("bits", C.c_void_p),
+        ("sched", C.c_void_p),
         ("n_groups", C.c_int64),
         ("union_cap", C.c_int64),
         ("words", C.c_int32),

@@ -55,6 +55,7 @@ class Groups:
     union_off: torch.Tensor
     union_pages: torch.Tensor
     bits: torch.Tensor
+    sched: torch.Tensor
     workspace: torch.Tensor
     n_groups: int
     union_cap: int
@@ -74,13 +75,15 @@ class Groups:
             union_off=torch.empty(ng + 1, **i32),
             union_pages=torch.empty(max(uc, 1), **i32),
             bits=torch.empty(max(T * Hkv * words, 1), dtype=torch.int32, device=device),
+            sched=torch.zeros(1, **i32),
             workspace=torch.empty(ws, dtype=torch.uint8, device=device),
             n_groups=ng, union_cap=uc, words=words, g=g, W=W)
 
     def struct(self) -> PwGroups:
         return PwGroups(self.qids.data_ptr(), self.gsize.data_ptr(), self.gmeta.data_ptr(),
                         self.union_off.data_ptr(), self.union_pages.data_ptr(),
-                        self.bits.data_ptr(), self.n_groups, self.union_cap, self.words, self.g)
+                        self.bits.data_ptr(), self.sched.data_ptr(), self.n_groups,
+                        self.union_cap, self.words, self.g)
 
     def to_host(self) -> dict:
         """Group arrays copied to the host, trimmed to n_groups and the union length."""

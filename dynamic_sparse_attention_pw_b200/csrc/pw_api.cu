@@ -64,7 +64,7 @@ size_t workspace_for(const Sizes &z, int Hkv)
 
 extern "C" {
 
-int pw_version(void) { return 100; }
+int pw_version(void) { return 101; }
 
 const char *pw_status_string(int s)
 {
@@ -172,7 +172,7 @@ pw_status pw_attn(const void *Q, const void *K_pages, const void *V_pages,
         return PW_ERR_INVALID_ARG;
     if (groups->n_groups > 0 &&
         (!Q || !K_pages || !V_pages || !page_table || !O || !groups->qids || !groups->gsize ||
-         !groups->gmeta || !groups->union_off || !groups->bits))
+         !groups->gmeta || !groups->union_off || !groups->bits || !groups->sched))
         return PW_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K_pages) |
          reinterpret_cast<uintptr_t>(V_pages) | reinterpret_cast<uintptr_t>(O)) & 15u)
@@ -199,6 +199,8 @@ pw_status pw_attn(const void *Q, const void *K_pages, const void *V_pages,
     L.union_off = groups->union_off;
     L.union_pages = groups->union_pages;
     L.bits = groups->bits;
+    L.sched = groups->sched;
+    L.dyn_sched = B > 1 ? 1 : 0;
     L.words = groups->words;
     L.g = groups->g;
     L.n_groups = groups->n_groups;

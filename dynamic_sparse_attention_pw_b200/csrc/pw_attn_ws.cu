@@ -12,8 +12,9 @@
 // O += P V runs on f16 operands with P read from TMEM: P split into f16 hi + lo parts, both
 // multiplied into the one accumulator, and V decoded exactly (E4M3 is a subset of f16).
 //
-// One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... .  A step is one or
-// two union pages of a group.  Its warps:
+// One CTA per SM walks the groups blockIdx.x, blockIdx.x + gridDim.x, ... (a ragged batch: takes
+// them from a work counter, the last group first, until none are left).  A step is one or two
+// union pages of a group.  Its warps:
 //   warps 0-3    decode   E4M3 V pages -> f16 operand tiles, one step at a time
 //   warps 4-11   softmax  S -> P for each step (four threads per row, 16 keys of each page each;
 //                         both pages' scores in one TMEM round trip), written back to TMEM over
@@ -546,6 +547,9 @@ __device__ __noinline__ SlowOut softmax_slow_path(WsSmem &sm, int row, int qq, i
 
 // tmap_k: the K pages as a 2-D byte tensor [n_phys * Hkv * 64 rows][128], boxes of 64 x 128
 // with the 128-byte swizzle, so that one copy lands a page as the K-major operand of S.
+// kDyn: groups from the launch's work counter (ragged batches) instead of a fixed stride; two
+// instantiations, so that each carries the code of one schedule only.
+template <bool kDyn>
 __global__ void __launch_bounds__(kThreads, 1)
     k_union_attn_ws(const AttnLaunch L, const __grid_constant__ CUtensorMap tmap_k)
 {
@@ -601,7 +605,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int64_t g0 = blockIdx.x, gstep = gridDim.x;
 
     if (warp == kWarpLoad) {
         // ---------------- load: group records, Q rows, union pages -> stages ----------------
@@ -615,16 +618,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             return __all_sync(kFull, wait_bar_c(bar, parity, &sm.abort_flag));
         };
         struct GMeta {
-            int64_t gi;
             int b, h, gsz, R, u0, nU, pg0, pg1, pg2, pg3;
             int32_t tok_l, cu_b;   // lane l: query l of the group
             uint32_t w0_l, w1_l;   // lane l: its membership words of the first two union pages
         };
-        // The next group with union pages, from gi on; groups without any get their zero rows.
-        // A record that would address outside the launch's buffers (sequence, head, size or a
-        // member token out of range) is skipped and recorded as PW_ERR_INVALID_ARG.
-        auto next_group = [&](int64_t gi, GMeta &m) -> bool {
-            for (; gi < L.n_groups; gi += gstep) {
+        // The next group with union pages; groups without any get their zero rows.  With
+        // kDyn (a ragged batch) groups come from the launch's work counter: ticket t is
+        // group n_groups - 1 - t, so the longest sequences' groups, which carry the largest
+        // unions, start first and short groups fill the end, and every CTA stays busy until
+        // the last tickets are gone (lane 0 holds the next ticket, taken one group early so
+        // that the atomic's round trip overlaps the current group's copies; a CTA never holds
+        // more than one unused ticket, and once one is past the last group so are all later
+        // ones).  Otherwise CTA i takes groups i, i + gridDim.x, ...: on a single sequence this
+        // measured faster than the counter.  A record that would address outside the launch's
+        // buffers (sequence, head, size or a member token out of range) is skipped and
+        // recorded as PW_ERR_INVALID_ARG.
+        int ticket = kDyn && lane == 0 ? atomicAdd(L.sched, 1) : 0;
+        int64_t g_static = blockIdx.x;
+        auto next_index = [&]() -> int64_t {
+            if (!kDyn) {
+                const int64_t gi = g_static;
+                g_static += gridDim.x;
+                return gi < L.n_groups ? gi : -1;
+            }
+            const int t = __shfl_sync(kFull, ticket, 0);
+            if (t >= L.n_groups)
+                return -1;
+            if (lane == 0)
+                ticket = atomicAdd(L.sched, 1);
+            return L.n_groups - 1 - t;
+        };
+        auto next_group = [&](GMeta &m) -> bool {
+            for (;;) {
+                const int64_t gi = next_index();
+                if (gi < 0)
+                    return false;
                 const int b = L.gmeta[3 * gi], h = L.gmeta[3 * gi + 1];
                 const int gsz = L.gsize[gi], R = gsz * L.G;
                 const int u0 = L.union_off[gi], nU = L.union_off[gi + 1] - u0;
@@ -647,7 +675,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     continue;
                 }
-                m.gi = gi;
                 m.b = b;
                 m.h = h;
                 m.gsz = gsz;
@@ -665,7 +692,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m.w1_l = lane < gsz ? __ldg(bitrow + page_word(L, m.pg1)) : 0u;
                 return true;
             }
-            return false;
         };
         // Record of job n (or the end marker when m is null) into its ring slot.
         auto publish = [&](uint32_t n, const GMeta *m) -> bool {
@@ -719,12 +745,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, stp = 0;
         bool stop = false, has_cur = false;
         GMeta cur{}, nxt{};
-        int64_t gi_next = g0;
         // Iteration n publishes job n (the next group's record, or the end marker), then issues
         // the pages of job n - 1 and, as soon as the raw Q buffer is free, job n's Q rows.  One
         // call site for each keeps this role's code small.
         for (uint32_t n = 0; !stop; ++n) {
-            const bool has_nxt = next_group(gi_next, nxt);
+            const bool has_nxt = next_group(nxt);
             if (!publish(n, has_nxt ? &nxt : nullptr)) {
                 stop = true;
                 break;
@@ -788,7 +813,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             cur = nxt;
             has_cur = true;
-            gi_next = nxt.gi + gstep;
         }
     } else if (warp == kWarpMma || warp == kWarpPv) {
         // ---------------- MMA issue: two warps ----------------
@@ -1317,12 +1341,15 @@ cudaError_t attn_ws_launch(const AttnLaunch &L, cudaStream_t st)
     if (e != cudaSuccess)
         return e;
     const size_t smem = sizeof(WsSmem) + 1024;
-    e = cudaFuncSetAttribute(k_union_attn_ws, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = L.dyn_sched ? k_union_attn_ws<true> : k_union_attn_ws<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     if (e != cudaSuccess)
         return e;
     const int64_t grid = L.n_groups < sms ? L.n_groups : sms;
-    k_union_attn_ws<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(L, tmap_k);
+    if (L.dyn_sched && (e = cudaMemsetAsync(L.sched, 0, sizeof(int32_t), st)) != cudaSuccess)
+        return e;
+    kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(L, tmap_k);
     return cudaGetLastError();
 }
 

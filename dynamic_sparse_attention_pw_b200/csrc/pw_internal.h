@@ -41,6 +41,8 @@ struct AttnLaunch {
     float k_scale, v_scale, sm_scale;
     const int32_t *qids, *gsize, *gmeta, *union_off, *union_pages;
     const uint32_t *bits;
+    int32_t *sched;         // work counter of the persistent kernel, zeroed before its launch
+    int dyn_sched;          // take groups from sched (ragged batches) instead of a fixed stride
     int words, g;
     int64_t n_groups;
     uint16_t *O;            // bf16 bits

@@ -73,6 +73,11 @@ typedef enum pw_status {
  *   union_pages int32  [union_cap]     logical page ids of each group's union, ascending
  *   bits        uint32 [T * Hkv * words] page bitset of every (token, kv head) selection;
  *                                      pw_attn reads it for the per-query membership masks
+ *   sched       int32  [1]             scratch of pw_attn: for a batch of several sequences,
+ *                                      the work counter its CTAs take groups from (pw_attn
+ *                                      zeroes it on its stream before the kernel, so two
+ *                                      pw_attn calls on one pw_groups must not run at the same
+ *                                      time; pw_group does not touch it)
  * Groups are ordered by (b, h, w, seed token).
  */
 typedef struct pw_groups {
@@ -82,6 +87,7 @@ typedef struct pw_groups {
     int32_t *union_off;
     int32_t *union_pages;
     uint32_t *bits;
+    int32_t *sched;
     int64_t n_groups;
     int64_t union_cap;
     int32_t words;

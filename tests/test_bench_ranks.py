@@ -43,3 +43,16 @@ def test_two_gloo_ranks(tmp_path):
         assert r["ms"] == 8.0                       # the slowest rank's time, on every rank
         assert r["rate"] == pytest.approx(2.0e12 * 2 / 8e-3 / 1e12)
     assert res[1]["ref"] == 0                       # the reference arm: rank 1 exits without work
+
+
+def test_launch_count_follows_the_grouping_path():
+    """Five kernels per call, six when pw_group renumbers windows first (rows of more than 8
+    words that would take more than 2112 words of shared memory per warp staged whole)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.launches_per_call(32, 128) == 6   # 64K tokens, W = 128
+    assert bench.launches_per_call(32, 256) == 6
+    assert bench.launches_per_call(32, 64) == 5    # 32 x 65 = 2080 words: staged
+    assert bench.launches_per_call(16, 128) == 5   # 32K tokens: 16 x 129 = 2064 words
+    assert bench.launches_per_call(8, 256) == 5    # at most 8 words: always staged
+    assert bench.launches_per_call(1, 32) == 5

@@ -49,6 +49,8 @@ SMALL = [
     (_small(7, [2048], 8, 1, 32, "uniform"), 64, 8),
     # tile rows not a multiple of 32 and g not a power of two
     (_small(8, [450], 10, 2, 7, "community", communities=2), 30, 6),
+    # G = 4 with sixteen queries per group: a full 64-row tile on the pipelined kernel
+    (_small(18, [1500, 333], 8, 2, 10, "community", communities=4), 64, 16),
 ]
 
 
@@ -108,8 +110,8 @@ def test_attn_full_workload_every_row(cfg, W):
     parity.compare_rows(got.reshape(-1, 128), ref.reshape(-1, 128), wl.name)
 
 
-@pytest.mark.parametrize("cfg,W,g", [(3, 128, 8), (3, 8, 8), (3, 128, 1), (4, 128, 8),
-                                     (4, 256, 8), (5, 128, 8)])
+@pytest.mark.parametrize("cfg,W,g", [(3, 128, 8), (3, 8, 8), (3, 128, 1), (3, 128, 16),
+                                     (4, 128, 8), (4, 256, 8), (5, 128, 8)])
 def test_attn_full_workload_sampled_rows(cfg, W, g):
     wl = synth.WORKLOADS[cfg]
     inp = parity.inputs(wl)
