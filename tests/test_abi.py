@@ -7,7 +7,7 @@ import re
 import numpy as np
 import pytest
 
-from dynamic_sparse_attention_pw_b200 import _lib, build
+from dynamic_sparse_attention_pw_b200 import _lib, api, build
 from dynamic_sparse_attention_pw_b200 import synth
 from oracle import oracle
 
@@ -127,6 +127,26 @@ def test_calls_reject_bad_arguments_before_any_device_work(L):
                    C.c_void_p(16), 1, 128, 16, 2, 1.0, 1.0, 0.1, None, C.c_void_p(16),
                    C.c_void_p(16), None)
     assert st == _lib.PW_ERR_INVALID_ARG
+    # groups whose arrays are all given except the work counter
+    for f in ("qids", "gsize", "gmeta", "union_off", "union_pages", "bits"):
+        setattr(g, f, 256)
+    g.sched = None
+    st = L.pw_attn(C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), 2, 2,
+                   C.c_void_p(16), 1, 128, 16, 2, 1.0, 1.0, 0.1, C.byref(g), C.c_void_p(16),
+                   C.c_void_p(16), None)
+    assert st == _lib.PW_ERR_INVALID_ARG
+
+
+def test_device_status_codes_reach_the_caller_by_name():
+    """What a kernel records in the status word (a bounded wait that ran out, a bad selection,
+    an out-of-range page-table entry) is raised by check_status with the code's name."""
+    import torch
+    for code, word in ((_lib.PW_ERR_TIMEOUT, "wait"), (_lib.PW_ERR_BAD_SELECTION, "selected"),
+                       (_lib.PW_ERR_INVALID_ARG, "")):
+        with pytest.raises(_lib.PwError) as e:
+            api.check_status(torch.tensor([code], dtype=torch.int32), "test")
+        assert word in str(e.value).lower()
+    api.check_status(torch.zeros(1, dtype=torch.int32), "test")
 
 
 def test_product_path_has_no_fallback():
