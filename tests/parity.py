@@ -61,8 +61,9 @@ def sample_rows(wl: synth.Workload, groups: dict, n_random: int, seed: int = 0,
       - one row (random member, random head) of every group, so every group's union, page
         steps and odd page counts are exercised;
       - every row of the n_largest groups with the longest unions;
-      - every row of each persistent CTA's first and last group (the kernel walks the groups
-        gi, gi + n_ctas, ...), where its pipelines fill and drain;
+      - every row of the first and the last n_ctas groups: where the persistent kernel's CTAs
+        start and finish, both for a single sequence (CTA i walks i, i + n_ctas, ...) and for a
+        ragged batch (CTAs take groups from a counter, the last group first);
       - every row of the first, a middle and the last group;
       - n_random uniformly drawn rows."""
     rng = np.random.default_rng(seed)
