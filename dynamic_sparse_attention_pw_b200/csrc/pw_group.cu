@@ -3,10 +3,11 @@
 // paper, paper summary: greedy inside a bounded window, collecting queries whose selected sets
 // add few new pages, with the execution size g fixed independently of W).
 //
-// Four launches on the caller's stream:
+// Four or five launches on the caller's stream:
 //   k_bitsets        sel_pages -> per-(token, kv head) page bitsets + set sizes (validation)
-//   k_greedy_local   one warp per (sequence, kv head, window): the window's pages renumbered
-//                    densely, then the ballot/popcount greedy on the short rows
+//   k_greedy_local   (long sequences only) one warp per (sequence, kv head, window): the
+//                    window's pages renumbered densely, then the ballot/popcount greedy on the
+//                    short rows
 //   k_greedy<..>     the same greedy on rows of the sequence's length: short sequences, and
 //                    the windows whose page union is too large to renumber into 8 words
 //   k_union_offsets  exclusive scan of the union sizes -> CSR offsets
