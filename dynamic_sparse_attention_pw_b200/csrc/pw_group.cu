@@ -42,7 +42,8 @@ __device__ __forceinline__ int seq_of_token(const int32_t *cu, int B, int64_t t)
 // into per-head bitsets in shared memory and written out as hc contiguous rows.  Invalid ids
 // (outside [-1, own page]) are reported and skipped.  counts[t, h] = |S(t, h)| (distinct
 // pages).  When one load per lane and head covers a token (kmax <= 32, Hkv <= 8), the next
-// token's ids are loaded while the current one is built.
+// token's ids are loaded while the current one is built, and the set sizes are counted as the
+// bits are set.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void bitsets_fold(const int32_t *p, int nload, int hh, int own,
                                              int words, uint32_t *acc, int32_t *status)
@@ -88,11 +89,18 @@ __global__ void __launch_bounds__(256) k_bitsets(const int32_t *__restrict__ sel
     extern __shared__ uint32_t sh_acc[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
-    uint32_t *acc = sh_acc + wib * hc * words;
+    // per warp: hc bitset rows, then hc set-size counters, rounded up to 16 bytes
+    const int region = (hc * words + hc + 3) & ~3;
+    uint32_t *acc = sh_acc + wib * region;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + wib;
     if (kmax <= 32 && Hkv <= kLoads) {
-        // hc == Hkv here: one pass per token, its ids one load per lane and head
+        // hc == Hkv here: one pass per token, its ids one load per lane and head.  A set's size
+        // is counted as its bits are set (an id whose bit was clear adds one), and the rows go
+        // out as 16-byte vectors when they allow it.
+        const int nw = Hkv * words;
+        uint32_t *cnt = acc + nw;
+        const bool vec = (nw & 3) == 0 && (reinterpret_cast<uintptr_t>(bits) & 15) == 0;
         int32_t p[kLoads];
 #pragma unroll
         for (int u = 0; u < kLoads; ++u)
@@ -105,12 +113,39 @@ __global__ void __launch_bounds__(256) k_bitsets(const int32_t *__restrict__ sel
                 q[u] = tn < T && u < Hkv && lane < kmax ? sel[(tn * Hkv + u) * kmax + lane] : -1;
             const int b = seq_of_token(cu, B, t);
             const int own = static_cast<int>((t - cu[b]) >> 6);
-            for (int i = lane; i < Hkv * words; i += 32)
-                acc[i] = 0;
+            if (vec) {
+                for (int i = lane; i < (nw >> 2); i += 32)
+                    reinterpret_cast<uint4 *>(acc)[i] = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                for (int i = lane; i < nw; i += 32)
+                    acc[i] = 0;
+            }
+            if (lane < Hkv)
+                cnt[lane] = 0;
             __syncwarp();
-            bitsets_fold(p, Hkv, 0, own, words, acc, status);
+#pragma unroll
+            for (int u = 0; u < kLoads; ++u) {
+                if (u >= Hkv || p[u] == -1)
+                    continue;
+                if (p[u] < -1 || p[u] > own) {
+                    set_status(status, PW_ERR_BAD_SELECTION);
+                    continue;
+                }
+                const uint32_t bit = 1u << (p[u] & 31);
+                if ((atomicOr(&acc[u * words + (p[u] >> 5)], bit) & bit) == 0u)
+                    atomicAdd(&cnt[u], 1u);
+            }
             __syncwarp();
-            bitsets_emit(t, 0, Hkv, Hkv, words, lane, acc, bits, counts);
+            uint32_t *out = bits + static_cast<size_t>(t) * nw;
+            if (vec) {
+                for (int i = lane; i < (nw >> 2); i += 32)
+                    reinterpret_cast<uint4 *>(out)[i] = reinterpret_cast<const uint4 *>(acc)[i];
+            } else {
+                for (int i = lane; i < nw; i += 32)
+                    out[i] = acc[i];
+            }
+            if (lane < Hkv)
+                counts[static_cast<size_t>(t) * Hkv + lane] = static_cast<uint16_t>(cnt[lane]);
             __syncwarp();
 #pragma unroll
             for (int u = 0; u < kLoads; ++u)
@@ -934,7 +969,8 @@ cudaError_t group_launch(const GroupLaunch &L, cudaStream_t st)
         const int warps = 8;
         int hc = 512 / L.words; // heads per pass: at most 2 KiB of bitsets per warp
         hc = hc < 1 ? 1 : (hc > L.Hkv ? L.Hkv : hc);
-        const size_t smem = static_cast<size_t>(warps) * hc * L.words * sizeof(uint32_t);
+        const size_t smem = static_cast<size_t>(warps) * ((hc * L.words + hc + 3) & ~3) *
+                            sizeof(uint32_t);
         // one resident wave of warps striding over the tokens (each warp prefetches its next
         // token's ids)
         int dev = 0, sms = 0, per_sm = 0;
